@@ -1,0 +1,178 @@
+/*
+ * tq.h -- C ABI of libtq: the TurboQuant KV-cache codec and the fused decode
+ * attention that reads it, for NVIDIA B200 (sm_100a).
+ *
+ * What the operations are (cited by page title and section):
+ *  - "TurboQuant Performance Benefits: Memory Reduction and Speed Optimization
+ *    in MLX-VLM", sections "What Is TurboQuant?" and "Fractional-Bit Precision
+ *    Support": KV vectors are rotated with a random Hadamard transform, then
+ *    quantized with an MSE codebook to 2-4 bits per dimension; 3.5 bits means
+ *    3-bit keys and 4-bit values.
+ *  - same page, "Custom Metal Kernel Implementation": attention scores and the
+ *    value aggregation are computed directly on the packed codes during decode,
+ *    without dequantizing the cache.
+ *  - "How to Use TurboQuant with the MLX-VLM Python API: A Complete Guide",
+ *    section "What is TurboQuant?": the rotation helpers (_rotation_matrix,
+ *    _rht_forward, _rht_inverse) and the codebook generator (_codebook).
+ *  - "mlx-turboquant" README, section "The 1-bit QJL residual (unbiased
+ *    inner-product estimator)": keys may carry sign(RHT2(r)) and ||r|| of the
+ *    residual r = Rk - k_hat; the score adds
+ *    sqrt(pi/(2d)) * ||r|| * <RHT2(Rq), sign(RHT2(r))>.
+ *
+ * Conventions shared by every call:
+ *  - Pointers are plain host or device addresses as stated per argument; the
+ *    library never takes ownership of caller memory and never allocates device
+ *    memory.  The only object it allocates is the host-side tq_codebook.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Device work is enqueued on it and the call returns; results are
+ *    visible after the caller synchronizes that stream.
+ *  - A call that returns a status other than TQ_OK enqueued nothing, except
+ *    TQ_ERR_CUDA from a launch, which reports a failed launch.
+ *    tq_last_error() then describes the problem (thread-local string).
+ *  - Errors found on the device (a sequence that would pass the cache
+ *    capacity, a context longer than the decode call was sized for) never trap
+ *    and never wait: the kernel skips the affected work and ORs a TQ_FLAG_*
+ *    bit into *cache->status, which the caller reads after synchronizing.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID = 1,      /* bad argument: null pointer, size, alignment   */
+  TQ_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, bits, group    */
+  TQ_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed          */
+  TQ_ERR_CAPACITY = 4,     /* workspace too small                           */
+  TQ_ERR_NOMEM = 5         /* host allocation failed                        */
+} tq_status;
+
+/* Sticky device-side flags ORed into *tq_cache.status. */
+#define TQ_FLAG_CAPACITY 1u  /* an append would pass `capacity`: that batch row was skipped */
+#define TQ_FLAG_MAXCTX 2u    /* a sequence was longer than the decode's max_ctx: its tail was not attended */
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Codec parameters.
+ *   head_dim : d, one of 64, 128, 256
+ *   k_bits, v_bits : code widths in {2, 3, 4} ("3.5 bits" = 3 and 4)
+ *   qjl      : 1 = keys also carry the 1-bit QJL residual sketch
+ *   seed     : seeds the sign vectors of R (and of R2 = RHT2 for QJL).  One R
+ *              is shared by keys, values, all heads and all batch rows. */
+typedef struct {
+  int head_dim;
+  int k_bits;
+  int v_bits;
+  int qjl;
+  uint64_t seed;
+} tq_params;
+
+/* Bytes stored per cached vector, in each per-vector array of tq_cache. */
+typedef struct {
+  size_t k_code_bytes;   /* k_bits * head_dim / 8 */
+  size_t v_code_bytes;   /* v_bits * head_dim / 8 */
+  size_t k_sign_bytes;   /* head_dim / 8 with QJL, else 0 */
+} tq_layout;
+
+typedef struct tq_codebook tq_codebook;  /* opaque, host memory, owned by the library */
+
+/* The compressed cache: caller-owned DEVICE memory (e.g. torch tensors).
+ * Row r = b * kv_heads + h of every per-vector array holds `capacity` slots;
+ * slot t is token t of batch row b, KV head h.
+ *   k_codes : uint8 [batch][kv_heads][capacity][k_code_bytes]
+ *   v_codes : uint8 [batch][kv_heads][capacity][v_code_bytes]
+ *   k_signs : uint8 [batch][kv_heads][capacity][k_sign_bytes] (QJL only, else NULL)
+ *   k_norm, v_norm : fp16 bit patterns [batch][kv_heads][capacity] (||x||)
+ *   k_rnorm : fp16 bit patterns [batch][kv_heads][capacity] (QJL ||Rk - k_hat||, else NULL)
+ *   seq_lens : int32 [batch], tokens currently stored per batch row
+ *   status   : one int32, sticky TQ_FLAG_* bits (caller clears it)
+ *   append_sync : int32 [batch], zero before the first append; every
+ *                 tq_quantize_append leaves it zero again
+ * Packed code layout of one vector: a little-endian bit stream in which
+ * channel i's b-bit code occupies bits [b*i, b*i + b), bit 0 being the least
+ * significant bit of byte 0; the sign plane is the same stream with b = 1.
+ * capacity must be a multiple of 16.  Every pointer must be 16-byte aligned. */
+typedef struct {
+  uint8_t *k_codes, *v_codes, *k_signs;
+  uint16_t *k_norm, *v_norm, *k_rnorm;
+  int32_t *seq_lens;
+  int32_t *status;
+  int32_t *append_sync;
+  int batch, kv_heads, capacity;
+} tq_cache;
+
+/* Builds the codebooks and rotation signs for `params` (host work only: no
+ * GPU is needed).  Codebook: the Lloyd-Max MSE quantizer of N(0, 1) with
+ * 2^bits levels, solved in double precision, made exactly odd-symmetric and
+ * rounded to float32; boundaries are the float32 midpoints of adjacent
+ * centroids ("How to Use TurboQuant ...", "What is TurboQuant?": _codebook).
+ * Signs: channel i of D1 is -1 when the top bit of the i-th SplitMix64 output
+ * from state `seed` is set; D2 uses state seed ^ 0x9E3779B97F4A7C15.
+ * On success *out owns the tables (release with tq_free) and *layout, if not
+ * NULL, receives the per-vector byte counts. */
+tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout* layout);
+
+/* Copies the tables of `cb` into caller HOST buffers (any may be NULL):
+ * k_centroids[2^k_bits], k_boundaries[2^k_bits - 1], v_centroids[2^v_bits],
+ * v_boundaries[2^v_bits - 1], signs1[head_dim], signs2[head_dim] (+1/-1). */
+tq_status tq_codebook_tables(const tq_codebook* cb, float* k_centroids, float* k_boundaries,
+                             float* v_centroids, float* v_boundaries,
+                             int8_t* signs1, int8_t* signs2);
+
+/* Quantizes n_new new tokens per batch row and appends them at slots
+ * [seq_lens[b], seq_lens[b] + n_new), then adds n_new to seq_lens[b].
+ * k, v : DEVICE, dtype `dtype`, contiguous [batch][kv_heads][n_new][head_dim].
+ * Per vector x (fp32 arithmetic, fixed operation order, see the pages' codec):
+ *   n = ||x|| (pairwise sum of squares, correctly rounded sqrt), stored fp16;
+ *   u = H (s1 * x) (unnormalized Walsh-Hadamard, Sylvester order);
+ *   z = u * (1/n) (0 when n == 0);  code_i = #{j : boundary_j < z_i};
+ *   QJL keys: r = u - fp16(n) * c[code]; ||r||/sqrt(d) stored fp16;
+ *             sign bit_i = (H (s2 * r))_i >= 0.
+ * A batch row whose append would pass `capacity` is skipped and sets
+ * TQ_FLAG_CAPACITY.  n_new == 0 is a no-op.  NaN/Inf inputs are undefined; a
+ * norm above 65504 stores an infinite fp16 norm. */
+tq_status tq_quantize_append(const tq_codebook* cb, const tq_cache* cache, const void* k,
+                             const void* v, tq_dtype dtype, int n_new, void* stream);
+
+/* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes). */
+size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
+                                 int max_ctx);
+
+/* Decode attention of one new query per head over the compressed cache.
+ * q   : DEVICE, dtype `dtype`, [batch][q_heads][head_dim]; query head h reads
+ *       KV head h / (q_heads / kv_heads).
+ * out : DEVICE float32 [batch][q_heads][head_dim].
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ * max_ctx : host upper bound of every seq_lens[b] (at most capacity); it sizes
+ *       the split over the context.  Tokens past it are not attended and set
+ *       TQ_FLAG_MAXCTX.
+ * workspace : DEVICE scratch of at least
+ *       tq_decode_workspace_bytes(cb, batch, q_heads, kv_heads, max_ctx) bytes
+ *       (TQ_ERR_CAPACITY otherwise); it holds the per-split partial results.
+ * Computes, for every (b, h), over tokens t < seq_lens[b]:
+ *   s_t = scale * (<Rq, n_t c_K[code_t]/sqrt(d)>
+ *                  + sqrt(pi/(2d)) * rho_t * <R2 R q, 2 bit_t - 1>)   (QJL term if enabled)
+ *   out = R^T (sum_t softmax(s)_t * m_t c_V[vcode_t] / sqrt(d)),
+ * never writing a dequantized cache.  seq_lens[b] == 0 gives zeros.  The
+ * result is deterministic (fixed-order merge of the splits). */
+tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, const void* q,
+                              tq_dtype dtype, int q_heads, float softmax_scale, int max_ctx,
+                              float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Releases a codebook (NULL is ignored). */
+void tq_free(tq_codebook* cb);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

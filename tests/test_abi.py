@@ -1,0 +1,130 @@
+"""C-ABI checks that need no GPU: exports, host-side tables, argument validation."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from turboquant_kv_cache_rht_b200 import tq
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "tq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert set(names) == set(tq.EXPORTS)
+    for n in names:
+        assert hasattr(tq.lib, n), n
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb,vb", [(2, 2), (3, 4), (4, 4), (2, 3)])
+@pytest.mark.parametrize("seed", [0, 1234567, 2**64 - 1])
+def test_tables_equal_oracle_bit_for_bit(d, kb, vb, seed):
+    cb = tq.Codebook(d, kb, vb, qjl=True, seed=seed)
+    t = cb.tables()
+    for bits, c_name, b_name in ((kb, "k_centroids", "k_boundaries"), (vb, "v_centroids", "v_boundaries")):
+        cent, bnd = o.codebook(bits)
+        assert np.array_equal(t[c_name].numpy().view(np.uint32), cent.view(np.uint32))
+        assert np.array_equal(t[b_name].numpy().view(np.uint32), bnd.view(np.uint32))
+    assert np.array_equal(t["signs1"].numpy(), o.rotation_signs(seed, d))
+    assert np.array_equal(t["signs2"].numpy(), o.rotation_signs(seed, d, second=True))
+
+
+def test_layout_bytes():
+    cb = tq.Codebook(128, 3, 4, qjl=True)
+    assert (cb.layout.k_code_bytes, cb.layout.v_code_bytes, cb.layout.k_sign_bytes) == (48, 64, 16)
+    cb = tq.Codebook(256, 2, 2, qjl=False)
+    assert (cb.layout.k_code_bytes, cb.layout.v_code_bytes, cb.layout.k_sign_bytes) == (64, 64, 0)
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=96), dict(head_dim=512), dict(k_bits=1),
+                                 dict(v_bits=5), dict(qjl=2)])
+def test_codebook_rejects_bad_params(bad):
+    p = dict(head_dim=128, k_bits=3, v_bits=4, qjl=0, seed=0)
+    p.update(bad)
+    params = tq.tq_params(p["head_dim"], p["k_bits"], p["v_bits"], p["qjl"], p["seed"])
+    h = C.c_void_p()
+    assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_ERR_INVALID
+    assert not h.value
+    assert tq.tq_last_error()
+
+
+def test_head_dim_64_reported_unsupported():
+    params = tq.tq_params(64, 3, 4, 0, 0)
+    h = C.c_void_p()
+    assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_ERR_UNSUPPORTED
+
+
+def _fake_cache(batch=2, kv_heads=2, capacity=64, qjl=False, **over):
+    """A tq_cache struct with aligned fake addresses: validation reads no memory."""
+    a = iter(range(1 << 20, 1 << 30, 1 << 16))
+    c = tq.tq_cache(next(a), next(a), next(a) if qjl else None, next(a), next(a),
+                    next(a) if qjl else None, next(a), next(a), next(a), batch, kv_heads, capacity)
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def _append(cb, cache, n_new=1, k=1 << 12, v=1 << 13, dtype=1):
+    return tq.lib.tq_quantize_append(cb.handle, C.byref(cache), k, v, dtype, n_new, None)
+
+
+def test_append_validation():
+    cb = tq.Codebook(128, 3, 4)
+    assert _append(cb, _fake_cache(capacity=40)) == tq.TQ_ERR_INVALID      # not a multiple of 16
+    assert "multiple of 16" in tq.tq_last_error()
+    assert _append(cb, _fake_cache(k_codes=None)) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(k_norm=(1 << 20) + 2)) == tq.TQ_ERR_INVALID   # misaligned
+    assert _append(cb, _fake_cache(batch=0)) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(), n_new=-1) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(), dtype=7) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(), k=0) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(), k=(1 << 12) + 4) == tq.TQ_ERR_INVALID
+    assert _append(cb, _fake_cache(), n_new=0) == tq.TQ_OK                 # no-op, no launch
+    qcb = tq.Codebook(128, 3, 4, qjl=True)
+    assert _append(qcb, _fake_cache()) == tq.TQ_ERR_INVALID                # QJL needs k_signs
+    assert tq.lib.tq_quantize_append(None, C.byref(_fake_cache()), 1 << 12, 1 << 13, 1, 1,
+                                     None) == tq.TQ_ERR_INVALID
+
+
+def _decode(cb, cache, q_heads=4, max_ctx=64, ws=1 << 14, ws_bytes=1 << 30, scale=0.0, q=1 << 12):
+    return tq.lib.tq_decode_attention(cb.handle, C.byref(cache), q, 1, q_heads, scale, max_ctx,
+                                      1 << 13, ws, ws_bytes, None)
+
+
+def test_decode_validation():
+    cb = tq.Codebook(128, 3, 4)
+    assert _decode(cb, _fake_cache(), q_heads=3) == tq.TQ_ERR_INVALID       # not a multiple
+    assert _decode(cb, _fake_cache(), max_ctx=65) == tq.TQ_ERR_INVALID      # past capacity
+    assert _decode(cb, _fake_cache(), ws_bytes=16) == tq.TQ_ERR_CAPACITY
+    assert _decode(cb, _fake_cache(), q=0) == tq.TQ_ERR_INVALID
+    assert _decode(cb, _fake_cache(), scale=float("nan")) == tq.TQ_ERR_INVALID
+    assert _decode(cb, _fake_cache(kv_heads=1), q_heads=3) == tq.TQ_ERR_UNSUPPORTED   # group 3
+    assert _decode(cb, _fake_cache(kv_heads=1), q_heads=16) == tq.TQ_ERR_UNSUPPORTED  # group 16
+    cb35 = tq.Codebook(128, 4, 2)
+    assert _decode(cb35, _fake_cache()) == tq.TQ_ERR_UNSUPPORTED           # v_bits < k_bits
+
+
+def test_workspace_size_formula():
+    cb = tq.Codebook(128, 3, 4)
+    ws = tq.tq_decode_workspace_bytes(cb, 1, 32, 8, 32768)
+    assert ws > 0 and ws % (130 * 4 * 32) == 0
+    splits = ws // (130 * 4 * 32)
+    assert 1 <= splits <= 512 and splits * 8 >= 148       # at least one wave of CTAs
+    assert tq.tq_decode_workspace_bytes(cb, 1, 30, 8, 100) == 0
+    assert tq.tq_decode_workspace_bytes(cb, 32, 32, 8, 65536) % (130 * 4 * 32 * 32) == 0
+
+
+def test_kv_bits_split_matches_oracle():
+    for b in (2, 2.5, 3, 3.5, 4):
+        assert tq.kv_bits_split(b) == o.kv_bits_split(b)

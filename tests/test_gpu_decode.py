@@ -1,0 +1,143 @@
+"""GPU decode parity: tq_decode_attention through the C ABI vs the CPU oracle.
+
+The oracle encodes the same seeded raw K/V itself (codes are bit-exact, see
+test_gpu_codec) and computes attention in float64; the GPU result must satisfy,
+for every (batch row, query head), max |gpu - oracle| <= 2e-3 * max |oracle|.
+Covers several tiles plus a ragged tail, lengths 0/1/127/128/129, all GQA
+groups, both head dims, every bit pair, QJL, custom softmax scale, repeat-run
+determinism, independence of the split count, and the max_ctx flag.
+"""
+import numpy as np
+import pytest
+import torch
+
+from tests.tq_helpers import assert_rows_close, oracle_decode_unit, oracle_encode_unit, oracle_tables
+
+pytestmark = pytest.mark.gpu
+
+tq = pytest.importorskip("turboquant_kv_cache_rht_b200.tq")
+
+
+def _setup(d, kb, vb, qjl, B, Hkv, G, lengths, capacity, seed=7, dtype=torch.bfloat16,
+           corr=False):
+    g = torch.Generator().manual_seed(seed)
+    T = max(lengths)
+    k = torch.randn(B, Hkv, T, d, generator=g)
+    v = torch.randn(B, Hkv, T, d, generator=g)
+    k[..., 3] *= 20.0
+    v[..., 9] *= 20.0
+    q = torch.randn(B, Hkv * G, d, generator=g)
+    if corr:   # a few keys strongly aligned with a query head: peaked softmax
+        for b in range(B):
+            for h in range(Hkv):
+                for t in range(0, lengths[b], 97):
+                    k[b, h, t] = q[b, h * G + (t % G)] * 1.5
+    k, v, q = k.to(dtype), v.to(dtype), q.to(dtype)
+    cb = tq.Codebook(d, kb, vb, qjl, seed=seed)
+    cache = tq.Cache(cb, B, Hkv, capacity, "cuda")
+    # append the longest length for every row, then shorten rows to their own
+    # length: decode attends only slots below seq_lens[b]
+    if T > 0:
+        tq.tq_quantize_append(cb, cache, k.cuda(), v.cuda())
+    cache.seq_lens.copy_(torch.tensor(lengths, dtype=torch.int32))
+    torch.cuda.synchronize()
+    return cb, cache, k, v, q
+
+
+def _oracle(d, kb, vb, qjl, seed, k, v, q, lengths, G, scale=None):
+    tb = oracle_tables(d, kb, vb, qjl, seed)
+    B, Hkv = k.shape[0], k.shape[1]
+    out = np.zeros((B, Hkv * G, d))
+    for b in range(B):
+        for h in range(Hkv):
+            n = lengths[b]
+            ek, ev = oracle_encode_unit(tb, k[b, h, :n], v[b, h, :n])
+            out[b, h * G:(h + 1) * G] = oracle_decode_unit(tb, q[b, h * G:(h + 1) * G], ek, ev, scale)
+    return out
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb,vb,qjl", [(3, 4, False), (3, 4, True), (2, 2, True), (4, 4, False),
+                                       (2, 3, False), (3, 3, True)])
+def test_decode_matches_oracle(d, kb, vb, qjl):
+    G, B, Hkv = 4, 2, 2
+    lengths = [300, 129]
+    cb, cache, k, v, q = _setup(d, kb, vb, qjl, B, Hkv, G, lengths, 320, seed=kb * 10 + vb)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=320)
+    torch.cuda.synchronize()
+    ref = _oracle(d, kb, vb, qjl, kb * 10 + vb, k, v, q, lengths, G)
+    assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_gqa_groups(G):
+    d, B, Hkv = 128, 1, 2
+    lengths = [517]
+    cb, cache, k, v, q = _setup(d, 3, 4, True, B, Hkv, G, lengths, 528, seed=G, corr=True)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=528)
+    torch.cuda.synchronize()
+    ref = _oracle(d, 3, 4, True, G, k, v, q, lengths, G)
+    assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
+
+
+def test_edge_lengths_and_empty():
+    d, G, Hkv = 128, 4, 1
+    lengths = [1, 127, 128, 129, 0, 255, 256, 16]
+    B = len(lengths)
+    cb, cache, k, v, q = _setup(d, 3, 4, False, B, Hkv, G, lengths, 256, seed=3, dtype=torch.float32)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=256).cpu().numpy()
+    ref = _oracle(d, 3, 4, False, 3, k, v, q, lengths, G)
+    for b in range(B):
+        if lengths[b] == 0:
+            assert np.all(out[b] == 0)
+        else:
+            assert_rows_close(out[b], ref[b], what=f"len {lengths[b]}")
+
+
+def test_softmax_scale_and_fp32_query():
+    d, G, B, Hkv = 256, 2, 1, 3
+    lengths = [200]
+    cb, cache, k, v, q = _setup(d, 2, 3, True, B, Hkv, G, lengths, 208, seed=4, dtype=torch.float32)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), softmax_scale=0.3, max_ctx=208)
+    ref = _oracle(d, 2, 3, True, 4, k, v, q, lengths, G, scale=0.3)
+    assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
+
+
+def test_deterministic_and_split_independent():
+    d, G, B, Hkv = 128, 2, 4, 8
+    lengths = [3000, 2500, 1, 2999]
+    cb, cache, k, v, q = _setup(d, 3, 4, True, B, Hkv, G, lengths, 8192, seed=8)
+    qd = q.cuda()
+    a = tq.tq_decode_attention(cb, cache, qd, max_ctx=3000)
+    b = tq.tq_decode_attention(cb, cache, qd, max_ctx=3000)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)                                  # bit-identical reruns
+    c = tq.tq_decode_attention(cb, cache, qd, max_ctx=8192)   # another split of the context
+    ws1 = tq.tq_decode_workspace_bytes(cb, B, Hkv * G, Hkv, 3000) // (B * Hkv * G * (d + 2) * 4)
+    ws2 = tq.tq_decode_workspace_bytes(cb, B, Hkv * G, Hkv, 8192) // (B * Hkv * G * (d + 2) * 4)
+    assert (3000 + ws1 - 1) // ws1 != (8192 + ws2 - 1) // ws2   # different chunk lengths
+    rel = ((a - c).abs().amax(-1) / a.abs().amax(-1)).max().item()
+    assert rel <= 1e-5
+    tb = oracle_tables(d, 3, 4, True, 8)
+    for bb, h in ((0, 0), (3, 7), (2, 1)):
+        n = lengths[bb]
+        ek, ev = oracle_encode_unit(tb, k[bb, h, :n], v[bb, h, :n])
+        ref = oracle_decode_unit(tb, q[bb, h * G:(h + 1) * G], ek, ev)
+        assert_rows_close(a[bb, h * G:(h + 1) * G].cpu().numpy(), ref)
+
+
+def test_max_ctx_too_small_sets_flag():
+    d, G, B, Hkv = 128, 1, 1, 1
+    cb, cache, k, v, q = _setup(d, 3, 4, False, B, Hkv, G, [300], 512, seed=2)
+    tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=128)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) & tq.TQ_FLAG_MAXCTX
+
+
+def test_workspace_too_small_is_rejected():
+    d = 128
+    cb, cache, k, v, q = _setup(d, 3, 4, False, 1, 1, 1, [64], 64, seed=2)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=64,
+                               workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == tq.TQ_ERR_CAPACITY

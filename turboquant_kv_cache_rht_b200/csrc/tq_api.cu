@@ -1,0 +1,301 @@
+// C ABI of libtq: argument validation, codebook/sign construction on the host,
+// and kernel dispatch.  See include/tq.h for the contract of every entry point.
+#include "../../include/tq.h"
+#include "tq_internal.cuh"
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+struct tq_codebook {
+  tq_params params;
+  tq::Tables tables;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tq_status fail(tq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+tq_status ok() {
+  g_last_error.clear();
+  return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Lloyd-Max quantizer of the standard normal distribution ("How to Use
+// TurboQuant with the MLX-VLM Python API", "What is TurboQuant?": _codebook;
+// "mlx-turboquant" README: Lloyd-Max codebook for the near-Gaussian rotated
+// coordinates).  Lloyd's two conditions are iterated in double precision until
+// no level moves by 1e-14: boundaries at the midpoints of adjacent levels,
+// levels at the conditional means of their cells.
+// ---------------------------------------------------------------------------
+double normal_density(double x) {
+  if (std::isinf(x)) return 0.0;
+  return std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI);
+}
+
+// P(X > x)
+double normal_tail(double x) { return 0.5 * std::erfc(x / std::sqrt(2.0)); }
+
+// P(lo < X < hi), arranged so that neither tail is obtained by cancellation.
+double normal_mass(double lo, double hi) {
+  if (lo >= 0.0) return normal_tail(lo) - normal_tail(hi);
+  if (hi <= 0.0) return normal_tail(-hi) - normal_tail(-lo);
+  return 1.0 - normal_tail(-lo) - normal_tail(hi);
+}
+
+bool lloyd_max(int levels, double* level_out) {
+  double lv[16], next[16], edge[17];
+  for (int j = 0; j < levels; ++j) lv[j] = -2.0 + 4.0 * (j + 0.5) / levels;
+  for (int iter = 0; iter < 1000000; ++iter) {
+    edge[0] = -INFINITY;
+    edge[levels] = INFINITY;
+    for (int j = 1; j < levels; ++j) edge[j] = 0.5 * (lv[j - 1] + lv[j]);
+    double moved = 0.0;
+    for (int j = 0; j < levels; ++j) {
+      next[j] = (normal_density(edge[j]) - normal_density(edge[j + 1])) /
+                normal_mass(edge[j], edge[j + 1]);
+      moved = std::fmax(moved, std::fabs(next[j] - lv[j]));
+    }
+    std::memcpy(lv, next, sizeof(double) * levels);
+    if (moved < 1e-14) {
+      std::memcpy(level_out, lv, sizeof(double) * levels);
+      return true;
+    }
+  }
+  return false;
+}
+
+// float32 table: odd-symmetric levels, boundaries = float32 midpoints.
+bool build_codebook(int bits, float* cent, float* bnd) {
+  const int levels = 1 << bits, half = levels / 2;
+  double lv[16];
+  if (!lloyd_max(levels, lv)) return false;
+  for (int j = 0; j < half; ++j) {
+    const float pos = (float)((lv[half + j] - lv[half - 1 - j]) / 2.0);
+    cent[half + j] = pos;
+    cent[half - 1 - j] = -pos;
+  }
+  for (int j = 0; j + 1 < levels; ++j) {
+    volatile float s = cent[j] + cent[j + 1];  // two float32 roundings, no contraction
+    bnd[j] = s * 0.5f;
+  }
+  for (int j = levels - 1; j < 16; ++j) bnd[j] = INFINITY;
+  for (int j = levels; j < 16; ++j) cent[j] = 0.0f;
+  return true;
+}
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the sign of channel i is the
+// top bit of the i-th output.
+void build_signs(uint64_t state, int d, uint32_t* mask) {
+  for (int w = 0; w < 8; ++w) mask[w] = 0;
+  for (int i = 0; i < d; ++i) {
+    state += 0x9E3779B97F4A7C15ull;
+    uint64_t z = state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    if (z >> 63) mask[i >> 5] |= 1u << (i & 31);
+  }
+}
+
+tq_status check_params(const tq_params* p) {
+  if (!p) return fail(TQ_ERR_INVALID, "params is NULL");
+  if (p->head_dim != 128 && p->head_dim != 256)
+    return fail(p->head_dim == 64 ? TQ_ERR_UNSUPPORTED : TQ_ERR_INVALID,
+                "head_dim %d: supported values are 128 and 256", p->head_dim);
+  if (p->k_bits < 2 || p->k_bits > 4 || p->v_bits < 2 || p->v_bits > 4)
+    return fail(TQ_ERR_INVALID, "k_bits=%d v_bits=%d: each must be 2, 3 or 4", p->k_bits,
+                p->v_bits);
+  if (p->qjl != 0 && p->qjl != 1) return fail(TQ_ERR_INVALID, "qjl must be 0 or 1");
+  return TQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tq_status check_cache(const tq_codebook* cb, const tq_cache* c) {
+  if (!cb) return fail(TQ_ERR_INVALID, "codebook is NULL");
+  if (!c) return fail(TQ_ERR_INVALID, "cache is NULL");
+  if (c->batch <= 0 || c->kv_heads <= 0 || c->capacity <= 0)
+    return fail(TQ_ERR_INVALID, "cache sizes must be positive (batch=%d kv_heads=%d capacity=%d)",
+                c->batch, c->kv_heads, c->capacity);
+  if (c->capacity % 16 != 0)
+    return fail(TQ_ERR_INVALID, "capacity %d is not a multiple of 16", c->capacity);
+  const void* need[] = {c->k_codes, c->v_codes, c->k_norm, c->v_norm, c->seq_lens, c->status,
+                        c->append_sync};
+  const char* names[] = {"k_codes", "v_codes", "k_norm", "v_norm", "seq_lens", "status",
+                         "append_sync"};
+  for (int i = 0; i < 7; ++i) {
+    if (!need[i]) return fail(TQ_ERR_INVALID, "cache.%s is NULL", names[i]);
+    if (i < 4 && !aligned16(need[i]))
+      return fail(TQ_ERR_INVALID, "cache.%s is not 16-byte aligned", names[i]);
+  }
+  if (cb->params.qjl) {
+    if (!c->k_signs || !c->k_rnorm)
+      return fail(TQ_ERR_INVALID, "QJL codebook needs cache.k_signs and cache.k_rnorm");
+    if (!aligned16(c->k_signs) || !aligned16(c->k_rnorm))
+      return fail(TQ_ERR_INVALID, "cache.k_signs / k_rnorm are not 16-byte aligned");
+  }
+  const double slots = (double)c->batch * c->kv_heads * c->capacity;
+  if (slots * 128.0 > 9.0e18) return fail(TQ_ERR_INVALID, "cache too large");
+  return TQ_OK;
+}
+
+tq::CacheView view_of(const tq_cache* c) {
+  tq::CacheView v;
+  v.k_codes = c->k_codes;
+  v.v_codes = c->v_codes;
+  v.k_signs = c->k_signs;
+  v.k_norm = c->k_norm;
+  v.v_norm = c->v_norm;
+  v.k_rnorm = c->k_rnorm;
+  v.seq_lens = c->seq_lens;
+  v.status = c->status;
+  v.append_sync = c->append_sync;
+  v.batch = c->batch;
+  v.kv_heads = c->kv_heads;
+  v.capacity = c->capacity;
+  return v;
+}
+
+tq_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout* layout) {
+  if (!out) return fail(TQ_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  tq_status st = check_params(params);
+  if (st != TQ_OK) return st;
+  tq_codebook* cb = new (std::nothrow) tq_codebook;
+  if (!cb) return fail(TQ_ERR_NOMEM, "host allocation of the codebook failed");
+  std::memset(cb, 0, sizeof *cb);
+  cb->params = *params;
+  tq::Tables& t = cb->tables;
+  t.d = params->head_dim;
+  t.k_bits = params->k_bits;
+  t.v_bits = params->v_bits;
+  t.qjl = params->qjl;
+  if (!build_codebook(params->k_bits, t.k_cent, t.k_bnd) ||
+      !build_codebook(params->v_bits, t.v_cent, t.v_bnd)) {
+    delete cb;
+    return fail(TQ_ERR_INVALID, "Lloyd-Max iteration did not converge");
+  }
+  build_signs(params->seed, params->head_dim, t.s1);
+  build_signs(params->seed ^ 0x9E3779B97F4A7C15ull, params->head_dim, t.s2);
+  if (layout) {
+    layout->k_code_bytes = (size_t)params->k_bits * params->head_dim / 8;
+    layout->v_code_bytes = (size_t)params->v_bits * params->head_dim / 8;
+    layout->k_sign_bytes = params->qjl ? (size_t)params->head_dim / 8 : 0;
+  }
+  *out = cb;
+  return ok();
+}
+
+tq_status tq_codebook_tables(const tq_codebook* cb, float* k_centroids, float* k_boundaries,
+                             float* v_centroids, float* v_boundaries, int8_t* signs1,
+                             int8_t* signs2) {
+  if (!cb) return fail(TQ_ERR_INVALID, "codebook is NULL");
+  const tq::Tables& t = cb->tables;
+  const int lk = 1 << t.k_bits, lv = 1 << t.v_bits;
+  if (k_centroids) std::memcpy(k_centroids, t.k_cent, sizeof(float) * lk);
+  if (k_boundaries) std::memcpy(k_boundaries, t.k_bnd, sizeof(float) * (lk - 1));
+  if (v_centroids) std::memcpy(v_centroids, t.v_cent, sizeof(float) * lv);
+  if (v_boundaries) std::memcpy(v_boundaries, t.v_bnd, sizeof(float) * (lv - 1));
+  for (int i = 0; i < t.d; ++i) {
+    if (signs1) signs1[i] = ((t.s1[i >> 5] >> (i & 31)) & 1u) ? -1 : 1;
+    if (signs2) signs2[i] = ((t.s2[i >> 5] >> (i & 31)) & 1u) ? -1 : 1;
+  }
+  return ok();
+}
+
+tq_status tq_quantize_append(const tq_codebook* cb, const tq_cache* cache, const void* k,
+                             const void* v, tq_dtype dtype, int n_new, void* stream) {
+  tq_status st = check_cache(cb, cache);
+  if (st != TQ_OK) return st;
+  if (n_new < 0) return fail(TQ_ERR_INVALID, "n_new %d is negative", n_new);
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (n_new == 0) return ok();
+  if (!k || !v) return fail(TQ_ERR_INVALID, "k or v is NULL");
+  if (n_new > cache->capacity)
+    return fail(TQ_ERR_INVALID, "n_new %d exceeds capacity %d", n_new, cache->capacity);
+  const size_t esz = dtype == TQ_F32 ? 4 : 2;
+  const size_t vec_bytes = esz * cb->params.head_dim;
+  if (((uintptr_t)k % vec_bytes) % 8 != 0 || ((uintptr_t)v % vec_bytes) % 8 != 0 ||
+      !aligned16(k) || !aligned16(v))
+    return fail(TQ_ERR_INVALID, "k and v must be 16-byte aligned");
+  return cuda_status(tq::launch_quantize_append(cb->tables, view_of(cache), k, v, (int)dtype,
+                                                n_new, (cudaStream_t)stream),
+                     "quantize-append launch");
+}
+
+size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
+                                 int max_ctx) {
+  if (!cb || batch <= 0 || q_heads <= 0 || kv_heads <= 0 || max_ctx < 0 ||
+      q_heads % kv_heads != 0)
+    return 0;
+  const tq::DecodePlan plan = tq::plan_decode(batch, kv_heads, max_ctx, cb->params.head_dim);
+  return tq::decode_workspace_bytes(plan, batch, q_heads, cb->params.head_dim);
+}
+
+tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, const void* q,
+                              tq_dtype dtype, int q_heads, float softmax_scale, int max_ctx,
+                              float* out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  tq_status st = check_cache(cb, cache);
+  if (st != TQ_OK) return st;
+  if (!q || !out) return fail(TQ_ERR_INVALID, "q or out is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (q_heads <= 0 || q_heads % cache->kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "q_heads %d is not a positive multiple of kv_heads %d", q_heads,
+                cache->kv_heads);
+  if (max_ctx < 0 || max_ctx > cache->capacity)
+    return fail(TQ_ERR_INVALID, "max_ctx %d outside [0, capacity %d]", max_ctx, cache->capacity);
+  if (!aligned16(q) || !aligned16(out))
+    return fail(TQ_ERR_INVALID, "q and out must be 16-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(TQ_ERR_INVALID, "softmax_scale is not finite");
+  const int d = cb->params.head_dim;
+  const int group = q_heads / cache->kv_heads;
+  if (!tq::decode_supported(d, group, cb->params.k_bits, cb->params.v_bits, cb->params.qjl))
+    return fail(TQ_ERR_UNSUPPORTED,
+                "no decode kernel for head_dim=%d group=%d k_bits=%d v_bits=%d qjl=%d "
+                "(group must be 1, 2, 4 or 8; v_bits must be k_bits or k_bits + 1)",
+                d, group, cb->params.k_bits, cb->params.v_bits, cb->params.qjl);
+  const tq::DecodePlan plan = tq::plan_decode(cache->batch, cache->kv_heads, max_ctx, d);
+  const size_t need = tq::decode_workspace_bytes(plan, cache->batch, q_heads, d);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(TQ_ERR_CAPACITY, "workspace of %zu bytes is smaller than the %zu needed",
+                workspace_bytes, need);
+  if (need > 0 && !aligned16(workspace))
+    return fail(TQ_ERR_INVALID, "workspace must be 16-byte aligned");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  return cuda_status(tq::launch_decode(cb->tables, view_of(cache), q, (int)dtype, q_heads, scale,
+                                       plan, out, (float*)workspace, (cudaStream_t)stream),
+                     "decode launch");
+}
+
+void tq_free(tq_codebook* cb) { delete cb; }
+
+const char* tq_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,14 @@
+// Decode-attention kernels for head_dim 128 (one translation unit per head_dim
+// so the build can compile them in parallel).
+#include "tq_decode_impl.cuh"
+
+namespace tq {
+
+template <>
+cudaError_t launch_decode_dim<128>(const Tables& tb, const CacheView& cv, const void* q, int dtype,
+                                  int q_heads, float scale_log2, const DecodePlan& plan, float* ws,
+                                  cudaStream_t stream) {
+  return dispatch_decode_dim<128>(tb, cv, q, dtype, q_heads, scale_log2, plan, ws, stream);
+}
+
+}  // namespace tq

@@ -1,0 +1,214 @@
+"""Python binding of libtq (ctypes).  Argument marshalling only.
+
+Every call below forwards to the C entry point of the same name in
+``include/tq.h``; all codec and attention work runs in the CUDA kernels of
+``libtq.so``.  PyTorch supplies device memory (the cache, inputs, outputs and
+workspace are torch tensors owned by the caller) and the current CUDA stream.
+
+Importing this module loads ``libtq.so`` from the package directory and raises
+ImportError if it has not been built (``python -m
+turboquant_kv_cache_rht_b200.build``); there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtq.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libtq.so is not built ({_LIB_PATH}); run "
+                      "`python -m turboquant_kv_cache_rht_b200.build`")
+lib = C.CDLL(_LIB_PATH)
+
+TQ_OK, TQ_ERR_INVALID, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_CAPACITY, TQ_ERR_NOMEM = range(6)
+TQ_FLAG_CAPACITY = 1
+TQ_FLAG_MAXCTX = 2
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append",
+           "tq_decode_workspace_bytes", "tq_decode_attention", "tq_free", "tq_last_error")
+
+
+class tq_params(C.Structure):
+    _fields_ = [("head_dim", C.c_int), ("k_bits", C.c_int), ("v_bits", C.c_int),
+                ("qjl", C.c_int), ("seed", C.c_uint64)]
+
+
+class tq_layout(C.Structure):
+    _fields_ = [("k_code_bytes", C.c_size_t), ("v_code_bytes", C.c_size_t),
+                ("k_sign_bytes", C.c_size_t)]
+
+
+class tq_cache(C.Structure):
+    _fields_ = [("k_codes", C.c_void_p), ("v_codes", C.c_void_p), ("k_signs", C.c_void_p),
+                ("k_norm", C.c_void_p), ("v_norm", C.c_void_p), ("k_rnorm", C.c_void_p),
+                ("seq_lens", C.c_void_p), ("status", C.c_void_p), ("append_sync", C.c_void_p),
+                ("batch", C.c_int), ("kv_heads", C.c_int), ("capacity", C.c_int)]
+
+
+lib.tq_codebook_init.argtypes = [C.POINTER(tq_params), C.POINTER(C.c_void_p), C.POINTER(tq_layout)]
+lib.tq_codebook_init.restype = C.c_int
+lib.tq_codebook_tables.argtypes = [C.c_void_p] + [C.c_void_p] * 6
+lib.tq_codebook_tables.restype = C.c_int
+lib.tq_quantize_append.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_void_p,
+                                   C.c_int, C.c_int, C.c_void_p]
+lib.tq_quantize_append.restype = C.c_int
+lib.tq_decode_workspace_bytes.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int]
+lib.tq_decode_workspace_bytes.restype = C.c_size_t
+lib.tq_decode_attention.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_int, C.c_int,
+                                    C.c_float, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t,
+                                    C.c_void_p]
+lib.tq_decode_attention.restype = C.c_int
+lib.tq_free.argtypes = [C.c_void_p]
+lib.tq_free.restype = None
+lib.tq_last_error.argtypes = []
+lib.tq_last_error.restype = C.c_char_p
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {tq_last_error()}")
+
+
+def tq_last_error() -> str:
+    return lib.tq_last_error().decode()
+
+
+def _check(st: int, where: str):
+    if st != TQ_OK:
+        raise TQError(st, where)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def kv_bits_split(kv_bits: float) -> tuple[int, int]:
+    """Key/value widths for a fractional kv_bits (3.5 -> 3-bit keys, 4-bit values)."""
+    return int(math.floor(kv_bits + 1e-9)), int(math.ceil(kv_bits - 1e-9))
+
+
+class Codebook:
+    """Owner of a tq_codebook handle (host memory; freed with tq_free)."""
+
+    def __init__(self, head_dim: int, k_bits: int, v_bits: int, qjl: bool = False, seed: int = 0):
+        self.params = tq_params(head_dim, k_bits, v_bits, int(bool(qjl)), seed & ((1 << 64) - 1))
+        self.layout = tq_layout()
+        h = C.c_void_p()
+        _check(lib.tq_codebook_init(C.byref(self.params), C.byref(h), C.byref(self.layout)),
+               "tq_codebook_init")
+        self.handle = h
+
+    @classmethod
+    def from_kv_bits(cls, head_dim: int, kv_bits: float, qjl: bool = False, seed: int = 0):
+        kb, vb = kv_bits_split(kv_bits)
+        return cls(head_dim, kb, vb, qjl, seed)
+
+    head_dim = property(lambda self: self.params.head_dim)
+    k_bits = property(lambda self: self.params.k_bits)
+    v_bits = property(lambda self: self.params.v_bits)
+    qjl = property(lambda self: bool(self.params.qjl))
+
+    def tables(self) -> dict:
+        """Host copies of the codebooks and rotation signs (tq_codebook_tables)."""
+        lk, lv, d = 1 << self.k_bits, 1 << self.v_bits, self.head_dim
+        kc, kb = (C.c_float * lk)(), (C.c_float * (lk - 1))()
+        vc, vb = (C.c_float * lv)(), (C.c_float * (lv - 1))()
+        s1, s2 = (C.c_int8 * d)(), (C.c_int8 * d)()
+        _check(lib.tq_codebook_tables(self.handle, kc, kb, vc, vb, s1, s2), "tq_codebook_tables")
+        to = lambda a, dt: torch.tensor(list(a), dtype=dt)
+        return {"k_centroids": to(kc, torch.float32), "k_boundaries": to(kb, torch.float32),
+                "v_centroids": to(vc, torch.float32), "v_boundaries": to(vb, torch.float32),
+                "signs1": to(s1, torch.int8), "signs2": to(s2, torch.int8)}
+
+    def __del__(self, _free=lib.tq_free):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            _free(h)
+            self.handle = None
+
+
+class Cache:
+    """A compressed KV cache held in torch tensors (the caller owns them)."""
+
+    def __init__(self, cb: Codebook, batch: int, kv_heads: int, capacity: int, device="cuda"):
+        lay = cb.layout
+        n = (batch, kv_heads, capacity)
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.batch, self.kv_heads, self.capacity = batch, kv_heads, capacity
+        self.k_codes = torch.zeros(*n, lay.k_code_bytes, **u8)
+        self.v_codes = torch.zeros(*n, lay.v_code_bytes, **u8)
+        self.k_signs = torch.zeros(*n, lay.k_sign_bytes, **u8) if cb.qjl else None
+        self.k_norm = torch.zeros(n, dtype=torch.float16, device=device)
+        self.v_norm = torch.zeros(n, dtype=torch.float16, device=device)
+        self.k_rnorm = torch.zeros(n, dtype=torch.float16, device=device) if cb.qjl else None
+        self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.append_sync = torch.zeros(batch, dtype=torch.int32, device=device)
+
+    def struct(self) -> tq_cache:
+        p = lambda t: None if t is None else t.data_ptr()
+        return tq_cache(p(self.k_codes), p(self.v_codes), p(self.k_signs), p(self.k_norm),
+                        p(self.v_norm), p(self.k_rnorm), p(self.seq_lens), p(self.status),
+                        p(self.append_sync), self.batch, self.kv_heads, self.capacity)
+
+    def nbytes(self) -> int:
+        ts = [self.k_codes, self.v_codes, self.k_signs, self.k_norm, self.v_norm, self.k_rnorm]
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return _DTYPES[t.dtype]
+
+
+def tq_quantize_append(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Tensor,
+                       stream=None) -> None:
+    """k, v: [batch, kv_heads, n_new, head_dim] contiguous CUDA tensors of one dtype."""
+    if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
+        raise ValueError("k and v must be [batch, kv_heads, n_new, head_dim] of one dtype")
+    if not (k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k and v must be contiguous")
+    if k.shape[0] != cache.batch or k.shape[1] != cache.kv_heads or k.shape[3] != cb.head_dim:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match the cache")
+    cs = cache.struct()
+    _check(lib.tq_quantize_append(cb.handle, C.byref(cs), k.data_ptr(), v.data_ptr(),
+                                  _dtype_code(k), k.shape[2], _stream_ptr(stream)),
+           "tq_quantize_append")
+
+
+def tq_decode_workspace_bytes(cb: Codebook, batch: int, q_heads: int, kv_heads: int,
+                              max_ctx: int) -> int:
+    return int(lib.tq_decode_workspace_bytes(cb.handle, batch, q_heads, kv_heads, max_ctx))
+
+
+def tq_decode_attention(cb: Codebook, cache: Cache, q: torch.Tensor, out: torch.Tensor | None = None,
+                        softmax_scale: float = 0.0, max_ctx: int | None = None,
+                        workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q: [batch, q_heads, head_dim] CUDA tensor; returns float32 [batch, q_heads, head_dim]."""
+    if q.dim() != 3 or q.shape[0] != cache.batch or q.shape[2] != cb.head_dim or not q.is_contiguous():
+        raise ValueError("q must be contiguous [batch, q_heads, head_dim]")
+    hq = q.shape[1]
+    max_ctx = cache.capacity if max_ctx is None else max_ctx
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    need = tq_decode_workspace_bytes(cb, cache.batch, hq, cache.kv_heads, max_ctx)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    cs = cache.struct()
+    _check(lib.tq_decode_attention(cb.handle, C.byref(cs), q.data_ptr(), _dtype_code(q), hq,
+                                   float(softmax_scale), int(max_ctx), out.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   _stream_ptr(stream)),
+           "tq_decode_attention")
+    return out
+
+
+def tq_free(cb: Codebook) -> None:
+    cb.__del__()
