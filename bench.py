@@ -1,0 +1,615 @@
+"""Benchmark of the TurboQuant decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa|qjl|long|serving|tiny]
+                    [--impl ours|reference] [--no-dense] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over one batch: tq_quantize_append of
+one new token per (batch row, KV head), then tq_decode_attention of every query
+head over the compressed cache.  Caches are pre-filled (bulk append, outside
+the timed region) with seeded synthetic K/V of the workload's shape.  Timing:
+W untimed warm-up steps, then exactly K steps between a barrier +
+synchronize on both sides, measured with CUDA events on the launching stream;
+steps rotate over cache replicas whose total size exceeds 4x L2, so every step
+reads its cache from HBM.  Steps are replayed from CUDA graphs (one per
+replica) so that host launch latency does not leak into the device time.
+
+The JSON line reports `value` = algorithmic bytes of the step (packed cache
+read by the decode, queries, outputs, appended K/V and their codes) / device
+time, in GB/s, plus ctx-tokens/s, the decode call's roofline against the
+measured HBM copy bandwidth, bulk quantize Mvec/s, an end-to-end figure through
+host buffers, the FP16/BF16 dense decode baselines on the same GPU, and the CPU
+oracle timed on the host as a baseline.
+
+With several GPUs (torchrun) every rank runs an independent replica of the
+workload ("replicas only": the path has no exchange step); `value` is the sum
+over ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from turboquant_kv_cache_rht_b200 import workloads as wl  # noqa: E402
+
+METRIC = "fused TQ decode-attention GB/s & % HBM peak; ctx-tokens/s; quantize Mvec/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# byte model (algorithmic bytes; see the design notes)
+# ---------------------------------------------------------------------------
+def token_bytes(w: wl.Workload) -> int:
+    """Packed bytes one decode reads per (token, KV head)."""
+    d = w.head_dim
+    b = w.k_bits * d // 8 + 2 + w.v_bits * d // 8 + 2
+    if w.qjl:
+        b += d // 8 + 2
+    return b
+
+
+def step_bytes(w: wl.Workload, lengths) -> dict:
+    esz = {"f32": 4, "bf16": 2, "f16": 2}[w.dtype]
+    d = w.head_dim
+    cache = sum(lengths) * w.kv_heads * token_bytes(w)
+    q_out = w.batch * w.q_heads * d * (esz + 4)
+    vec_out = (w.k_bits + w.v_bits) * d // 8 + 4 + ((d // 8 + 2) if w.qjl else 0)
+    append = w.batch * w.kv_heads * (2 * d * esz + vec_out)
+    return {"decode": cache + q_out, "append": append, "total": cache + q_out + append}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.out = None
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            sel = ["--id=" + bus] if bus else ["-i", "0"]
+        except Exception:
+            sel = ["-i", "0"]
+        self.cmd = ["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                    "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self) -> dict:
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for ln in self.out.strip().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, p in rows for i in range(4) if p[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+class State:
+    """Caches (replicas), per-step inputs and outputs of one workload on one GPU."""
+
+    def __init__(self, w: wl.Workload, steps_total: int, device):
+        from turboquant_kv_cache_rht_b200 import tq
+        self.tq = tq
+        self.w = w
+        self.dev = device
+        self.lengths = wl.context_lengths(w)
+        self.cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed)
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        per_replica = sum(self.lengths) * w.kv_heads * token_bytes(w)
+        self.replicas = max(1, math.ceil(4 * l2 / max(per_replica, 1)) + (0 if per_replica > 4 * l2 else 1))
+        self.replicas = min(self.replicas, 64)
+        visits = math.ceil(steps_total / self.replicas) + 8
+        self.capacity = (max(self.lengths) + visits + 15) // 16 * 16
+        self.max_ctx = max(self.lengths) + visits
+        self.caches = [tq.Cache(self.cb, w.batch, w.kv_heads, self.capacity, device)
+                       for _ in range(self.replicas)]
+        self._prefill()
+        self.q = wl.queries(w, 0).to(device)
+        kn, vn = wl.kv_step(w, 0)
+        self.k_new, self.v_new = kn.to(device).contiguous(), vn.to(device).contiguous()
+        self.out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float32, device=device)
+        ws = tq.tq_decode_workspace_bytes(self.cb, w.batch, w.q_heads, w.kv_heads, self.max_ctx)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+
+    def _prefill(self):
+        tq, w = self.tq, self.w
+        first = self.caches[0]
+        # bulk append one KV head at a time on the host side to bound host memory,
+        # then set each row's length (rows shorter than the longest keep zeros past it)
+        tmax = max(self.lengths)
+        for h in range(w.kv_heads):
+            kh = torch.zeros(w.batch, 1, tmax, w.head_dim, dtype=w.torch_dtype)
+            vh = torch.zeros_like(kh)
+            for b in range(w.batch):
+                k, v = wl.kv_unit(w, b, h, self.lengths[b])
+                kh[b, 0, :self.lengths[b]] = k
+                vh[b, 0, :self.lengths[b]] = v
+            tmp = tq.Cache(self.cb, w.batch, 1, self.capacity, self.dev)
+            tq.tq_quantize_append(self.cb, tmp, kh.to(self.dev), vh.to(self.dev))
+            for name in ("k_codes", "v_codes", "k_signs", "k_norm", "v_norm", "k_rnorm"):
+                src = getattr(tmp, name)
+                if src is not None:
+                    getattr(first, name)[:, h].copy_(src[:, 0])
+            del tmp
+        first.seq_lens.copy_(torch.tensor(self.lengths, dtype=torch.int32))
+        for c in self.caches[1:]:
+            for name in ("k_codes", "v_codes", "k_signs", "k_norm", "v_norm", "k_rnorm", "seq_lens"):
+                src = getattr(first, name)
+                if src is not None:
+                    getattr(c, name).copy_(src)
+        torch.cuda.synchronize(self.dev)
+
+    def step(self, r: int, stream=None):
+        tq = self.tq
+        c = self.caches[r]
+        tq.tq_quantize_append(self.cb, c, self.k_new, self.v_new, stream=stream)
+        tq.tq_decode_attention(self.cb, c, self.q, out=self.out, max_ctx=self.max_ctx,
+                               workspace=self.ws, stream=stream)
+
+
+def run_gpu(args, rank: int, world: int) -> dict | None:
+    import torch.distributed as dist
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = wl.WORKLOADS[args.workload]
+    K, W = args.steps, args.warmup
+    st = State(w, 2 * K + W, dev)
+    tq = st.tq
+    stream = torch.cuda.current_stream(dev)
+
+    # warm-up (also configures kernels before capture)
+    for i in range(W):
+        st.step(i % st.replicas)
+    torch.cuda.synchronize(dev)
+
+    graphs = []
+    cap_stream = torch.cuda.Stream(dev)
+    for r in range(st.replicas):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            st.step(r)
+        graphs.append(g)
+    torch.cuda.synchronize(dev)
+    for r in range(st.replicas):   # one graph replay each before timing
+        graphs[r].replay()
+    torch.cuda.synchronize(dev)
+
+    lengths_before = [int(x) for x in st.caches[0].seq_lens.cpu()]
+    visit = [0] * st.replicas
+    for r in range(st.replicas):
+        visit[r] = int(st.caches[r].seq_lens[0].item()) - st.lengths[0]
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda._sleep(2_000_000)          # let the host queue ahead of the device
+        e0.record(stream)
+        for s in range(K):
+            graphs[s % st.replicas].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    # bytes of the timed steps: replica r's contexts grew by one token per visit
+    total_bytes = 0
+    ctx_tokens = 0
+    for s in range(K):
+        r = s % st.replicas
+        grow = visit[r] + 1 + s // st.replicas
+        lens = [L + grow for L in st.lengths]
+        total_bytes += step_bytes(w, lens)["total"]
+        ctx_tokens += sum(lens)
+    ms_max = ms
+    bytes_all, tokens_all = float(total_bytes), float(ctx_tokens)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        t = torch.tensor([bytes_all, tokens_all], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        bytes_all, tokens_all = float(t[0].item()), float(t[1].item())
+
+    # ---- the decode call alone: events around each call, host queued ahead
+    dec_ms = []
+    app_ms = []
+    torch.cuda._sleep(2_000_000)
+    evs = []
+    for r in range(st.replicas):
+        a0, a1, d1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        c = st.caches[r]
+        a0.record(stream)
+        tq.tq_quantize_append(st.cb, c, st.k_new, st.v_new)
+        a1.record(stream)
+        tq.tq_decode_attention(st.cb, c, st.q, out=st.out, max_ctx=st.max_ctx, workspace=st.ws)
+        d1.record(stream)
+        evs.append((a0, a1, d1, [int(x) for x in st.lengths]))
+    torch.cuda.synchronize(dev)
+    for a0, a1, d1, _ in evs:
+        app_ms.append(a0.elapsed_time(a1))
+        dec_ms.append(a1.elapsed_time(d1))
+    dec_us = 1e3 * statistics.mean(dec_ms)
+    app_us = 1e3 * statistics.mean(app_ms)
+    lens_now = [int(x) for x in st.caches[0].seq_lens.cpu()]
+    dec_bytes = step_bytes(w, lens_now)["decode"]
+
+    # ---- bulk quantize throughput (prefill-style append of a whole context)
+    q_mvec = bulk_quantize_mvec(st, dev)
+
+    # ---- end to end through host buffers: pinned inputs in, result out, every step
+    e2e = end_to_end(st, dev, K, stream)
+
+    dense = None
+    if not args.no_dense and world == 1:
+        dense = dense_baselines(w, st, dev)
+
+    del graphs
+    peak, peak_kind = peaks()
+    achieved = dec_bytes / (dec_us * 1e-6) / 1e9
+    hbm_frac = achieved / peak
+    res = {
+        "metric": METRIC,
+        "value": round(bytes_all / (ms_max * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8 codes, f32 accumulate",
+        "data": "synthetic (seeded Gaussian K/V with outlier channels)",
+        "config": {"workload": w.name, "description": w.description, "batch": w.batch,
+                   "q_heads": w.q_heads, "kv_heads": w.kv_heads, "head_dim": w.head_dim,
+                   "context": st.lengths[0] if w.context else "ragged", "k_bits": w.k_bits,
+                   "v_bits": w.v_bits, "qjl": w.qjl, "parallelism": f"replicas x{world}",
+                   "l2": f"{st.replicas} rotating cache replicas "
+                         f"({st.replicas * sum(st.lengths) * w.kv_heads * token_bytes(w) / 1e6:.0f} MB, > 4x L2)"},
+        "ctx_tokens_per_s": round(tokens_all / (ms_max * 1e-3), 1),
+        "hbm_frac_of_step": round(bytes_all / (ms_max * 1e-3) / 1e9 / peak / world, 4),
+        "decode_us": round(dec_us, 3),
+        "append_us": round(app_us, 3),
+        "quantize_mvec_s": q_mvec,
+        "roofline": {"bound": "hbm", "kernel": "tq_decode_attention (decode + combine launches)",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(hbm_frac, 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": dec_bytes},
+        "e2e": e2e,
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+    if dense is not None:
+        res["dense_baseline"] = dense
+    return res
+
+
+def bulk_quantize_mvec(st: State, dev) -> dict:
+    """Append one full context of K/V (all heads) into a fresh cache; Mvec/s."""
+    tq, w = st.tq, st.w
+    n = min(max(st.lengths), 32768)
+    k, v = wl.kv_unit(w, 0, 0, n)
+    kk = k.to(dev)[None, None].expand(w.batch, w.kv_heads, n, w.head_dim).contiguous()
+    vv = v.to(dev)[None, None].expand(w.batch, w.kv_heads, n, w.head_dim).contiguous()
+    cap = (n + 15) // 16 * 16
+    c = tq.Cache(st.cb, w.batch, w.kv_heads, cap, dev)
+    times = []
+    for i in range(4):
+        c.seq_lens.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        tq.tq_quantize_append(st.cb, c, kk, vv)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        if i:
+            times.append(e0.elapsed_time(e1))
+    vecs = 2 * w.batch * w.kv_heads * n
+    ms = statistics.median(times)
+    esz = kk.element_size()
+    lay = st.cb.layout
+    byts = vecs // 2 * (2 * w.head_dim * esz + lay.k_code_bytes + lay.v_code_bytes + 4 +
+                        (lay.k_sign_bytes + 2 if w.qjl else 0))
+    return {"vectors": vecs, "ms": round(ms, 4), "mvec_s": round(vecs / (ms * 1e-3) / 1e6, 1),
+            "gb_s": round(byts / (ms * 1e-3) / 1e9, 1)}
+
+
+def end_to_end(st: State, dev, K: int, stream) -> dict:
+    """Same step through the public API with pinned host buffers copied in and out."""
+    tq, w = st.tq, st.w
+    hk = st.k_new.cpu().pin_memory()
+    hv = st.v_new.cpu().pin_memory()
+    hq = st.q.cpu().pin_memory()
+    hout = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
+    dk, dv, dq = torch.empty_like(st.k_new), torch.empty_like(st.v_new), torch.empty_like(st.q)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    tokens = 0
+    byts = 0
+    for s in range(K):
+        r = s % st.replicas
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        c = st.caches[r]
+        tq.tq_quantize_append(st.cb, c, dk, dv)
+        tq.tq_decode_attention(st.cb, c, dq, out=st.out, max_ctx=st.max_ctx, workspace=st.ws)
+        hout.copy_(st.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    lens = [int(x) for x in st.caches[0].seq_lens.cpu()]
+    byts = K * step_bytes(w, lens)["total"]
+    ms = e0.elapsed_time(e1)
+    h2d = hk.numel() * hk.element_size() + hv.numel() * hv.element_size() + hq.numel() * hq.element_size()
+    d2h = hout.numel() * hout.element_size()
+    return {"value": round(byts / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms / K, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def dense_baselines(w: wl.Workload, st: State, dev) -> dict:
+    """Unquantized bf16 decode attention on the same GPU: flash-attn's KV-cache
+    kernel and torch SDPA, on dense caches of the same shape (replicated past L2)."""
+    if w.batch * w.kv_heads * max(st.lengths) * w.head_dim * 2 * 2 > 40e9:
+        return {"skipped": "dense cache too large"}
+    res = {}
+    T = max(st.lengths)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    one = (torch.randn(w.batch, T, w.kv_heads, w.head_dim, generator=g)).to(torch.bfloat16).to(dev)
+    dense_bytes = one.numel() * 2 * 2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    reps = max(1, min(8, math.ceil(4 * l2 / dense_bytes) + 1)) if dense_bytes < 4 * l2 else 1
+    ks = [one] + [one.clone() for _ in range(reps - 1)]
+    vs = [one.clone() for _ in range(reps)]
+    q = st.q.to(torch.bfloat16).reshape(w.batch, 1, w.q_heads, w.head_dim)
+    seqlens = torch.tensor(st.lengths, dtype=torch.int32, device=dev)
+
+    def timeit(fn, n=20):
+        for i in range(3):
+            fn(i % reps)
+        torch.cuda.synchronize(dev)
+        torch.cuda._sleep(2_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            fn(i % reps)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return 1e3 * e0.elapsed_time(e1) / n
+
+    try:
+        from flash_attn import flash_attn_with_kvcache
+        res["flash_attn_us"] = round(timeit(lambda i: flash_attn_with_kvcache(
+            q, ks[i], vs[i], cache_seqlens=seqlens)), 2)
+    except Exception as e:  # library baseline only
+        res["flash_attn_error"] = repr(e)[:200]
+    try:
+        qs = q.transpose(1, 2).contiguous()
+        kt = [k.transpose(1, 2).contiguous() for k in ks]
+        vt = [v.transpose(1, 2).contiguous() for v in vs]
+        if len(set(st.lengths)) == 1:
+            res["sdpa_us"] = round(timeit(lambda i: torch.nn.functional.scaled_dot_product_attention(
+                qs, kt[i], vt[i], enable_gqa=True)), 2)
+    except Exception as e:
+        res["sdpa_error"] = repr(e)[:200]
+    times = [v for k, v in res.items() if k.endswith("_us")]
+    if times:
+        best = min(times)
+        res["best_dense_us"] = best
+        res["dense_bytes"] = dense_bytes
+        res["tq_decode_us"] = round(st_decode_us(st, dev), 2)
+        res["tq_speedup_vs_best_dense"] = round(best / res["tq_decode_us"], 3)
+    return res
+
+
+def st_decode_us(st: State, dev, n=None) -> float:
+    tq = st.tq
+    n = n or max(st.replicas, 8)
+    torch.cuda.synchronize(dev)
+    torch.cuda._sleep(2_000_000)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        tq.tq_decode_attention(st.cb, st.caches[i % st.replicas], st.q, out=st.out,
+                               max_ctx=st.max_ctx, workspace=st.ws)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    return 1e3 * e0.elapsed_time(e1) / n
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+class OracleUnit:
+    """One (batch row 0, KV head 0) unit of the workload, encoded by the oracle."""
+
+    def __init__(self, w: wl.Workload):
+        import numpy as np
+
+        import oracle as o
+        self.o, self.np, self.w = o, np, w
+        self.T = wl.context_lengths(w)[0]
+        d = w.head_dim
+        self.ck, self.bk = o.codebook(w.k_bits)
+        self.cv, self.bv = o.codebook(w.v_bits)
+        self.s1 = o.rotation_signs(w.rht_seed, d)
+        self.s2 = o.rotation_signs(w.rht_seed, d, second=True) if w.qjl else None
+        k, v = wl.kv_unit(w, 0, 0, self.T)
+        self.ek = o.encode(k.float().numpy(), self.s1, self.ck, self.bk, w.k_bits, self.s2)
+        self.ev = o.encode(v.float().numpy(), self.s1, self.cv, self.bv, w.v_bits)
+        kn, vn = wl.kv_step(w, 0)
+        self.k_new = kn[0, 0].float().numpy()
+        self.v_new = vn[0, 0].float().numpy()
+        self.q = wl.queries(w, 0)[0, :w.group].float().numpy().astype(np.float64)
+
+    def step(self):
+        """Append one token (encode K and V) and decode the unit's G heads."""
+        o, np, w = self.o, self.np, self.w
+        ek1 = o.encode(self.k_new, self.s1, self.ck, self.bk, w.k_bits, self.s2)
+        ev1 = o.encode(self.v_new, self.s1, self.cv, self.bv, w.v_bits)
+        kw = {}
+        if self.s2 is not None:
+            kw = dict(s2=self.s2, k_sign_bits=np.concatenate([self.ek["sign_bits"], ek1["sign_bits"]]),
+                      k_rnorm16=np.concatenate([self.ek["rnorm16"], ek1["rnorm16"]]))
+        return o.decode_attention(self.q, self.s1, np.concatenate([self.ek["idx"], ek1["idx"]]),
+                                  np.concatenate([self.ek["norm16"], ek1["norm16"]]), self.ck,
+                                  np.concatenate([self.ev["idx"], ev1["idx"]]),
+                                  np.concatenate([self.ev["norm16"], ev1["norm16"]]), self.cv, **kw)
+
+    def bytes_per_step(self) -> int:
+        w = self.w
+        esz = {"f32": 4, "bf16": 2, "f16": 2}[w.dtype]
+        d = w.head_dim
+        vec_out = (w.k_bits + w.v_bits) * d // 8 + 4 + ((d // 8 + 2) if w.qjl else 0)
+        return (self.T + 1) * token_bytes(w) + w.group * d * (esz + 4) + 2 * d * esz + vec_out
+
+
+def cpu_baseline(w: wl.Workload, budget_s: float = 12.0) -> dict:
+    u = OracleUnit(w)
+    u.step()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        u.step()
+        n += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or n >= 200:
+            break
+    return {"value": round(n * u.bytes_per_step() / el / 1e9, 4), "unit": "GB/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} steps of one (batch row, KV head) unit: encode 1 appended K and V, "
+                      f"decode {w.group} query heads over {u.T + 1} tokens (numpy, float64 attention)",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args, rank: int) -> dict | None:
+    if rank != 0:
+        return None
+    w = wl.WORKLOADS[args.workload]
+    u = OracleUnit(w)
+    for _ in range(args.warmup):
+        u.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        u.step()
+    el = time.perf_counter() - t0
+    value = args.steps * u.bytes_per_step() / el / 1e9
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 codec, f64 attention", "data": "synthetic",
+        "config": {"workload": w.name, "description": w.description,
+                   "sample": "one (batch row, KV head) unit of the workload per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: encode 1 appended K and V, decode {w.group} query heads "
+                                   f"over {u.T + 1} tokens of one KV head"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="gqa", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_gpu(args, rank, world)
+    if rank == 0 and res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl.WORKLOADS[args.workload])
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

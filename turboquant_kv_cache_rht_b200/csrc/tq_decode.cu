@@ -7,68 +7,143 @@ namespace tq {
 
 namespace {
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
 constexpr int kMaxSplits = 512;
 // Split target: about four CTAs per SM of a 148-SM B200.  Fixed (not queried)
 // so that the workspace size is a pure function of the call's sizes.
 constexpr long kTargetCtas = 148L * 4;
 
-// Merges the splits of one (query head, batch row) in split order and applies
-// the inverse rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
+// Merges the splits of one (query head, batch row) and applies the inverse
+// rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
 // w_s = 2^(m_s - max m) ("How to Use TurboQuant ...", "What is TurboQuant?":
 // _rht_inverse; the 1/d collects the rotation's and the dequantization's
-// 1/sqrt(d)).
+// 1/sqrt(d)).  Every partial is loaded at once (warp w takes splits w, w+8,
+// ..., lane l channels l*d/32 ..), so the merge costs one memory round trip;
+// all reductions run in a fixed order.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const __grid_constant__ Tables tb, const int32_t* __restrict__ seq_lens,
                    int32_t* status, const float* __restrict__ ws, int q_heads, int splits,
                    int chunk, int capacity, float* __restrict__ out) {
-  __shared__ float o[D];
+  constexpr int E = D / 32;
+  constexpr int W = kCombineThreads / 32;
+  constexpr int PER = 8;  // splits per warp per round, loaded together
   __shared__ float wgt[kMaxSplits];
-  __shared__ float inv_l;
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  __shared__ __align__(16) float part[W][D];
+  __shared__ float red[2][W];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  const long row = (long)b * q_heads + h;
+  const float* po = ws + row * splits * D;
+  const float* pml = ws + (long)gridDim.y * q_heads * splits * D + row * splits * 2;
+  // issue the loads of the first round before anything depends on them
+  float4 ov[PER][E / 4];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int s = warp + W * i;
+    if (s < splits) {
+#pragma unroll
+      for (int v = 0; v < E / 4; ++v)
+        ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * D + lane * E)[v];
+    }
+  }
+  float ms[kMaxSplits / kCombineThreads], ls[kMaxSplits / kCombineThreads];
+#pragma unroll
+  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i) {
+    const int s = tid + kCombineThreads * i;
+    ms[i] = s < splits ? pml[2 * s] : -INFINITY;
+    ls[i] = s < splits ? pml[2 * s + 1] : 0.f;
+  }
   const int T = min(max(seq_lens[b], 0), capacity);
   if (tid == 0 && h == 0 && T > (long)splits * chunk) atomicOr(status, (int)kFlagMaxCtx);
   const int S = min(splits, (T + chunk - 1) / chunk);
-  float* dst = out + ((long)b * q_heads + h) * D;
+  float* dst = out + row * D;
   if (S <= 0) {
     for (int i = tid; i < D; i += kCombineThreads) dst[i] = 0.f;
+    pdl_trigger();
     return;
   }
-  const float* src = ws + ((long)b * q_heads + h) * splits * (D + 2);
-  if (tid == 0) {
-    float m = -INFINITY;
-    for (int s = 0; s < S; ++s) m = fmaxf(m, src[(long)s * (D + 2)]);
-    float l = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float w = exp2f(src[(long)s * (D + 2)] - m);
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i)
+    if (tid + kCombineThreads * i < S) m = fmaxf(m, ms[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[0][warp] = m;
+  __syncthreads();
+  m = red[0][0];
+#pragma unroll
+  for (int w = 1; w < W; ++w) m = fmaxf(m, red[0][w]);
+  float l = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i) {
+    const int s = tid + kCombineThreads * i;
+    if (s < S) {
+      const float w = exp2f(ms[i] - m);
       wgt[s] = w;
-      l = fmaf(src[(long)s * (D + 2) + 1], w, l);
-    }
-    inv_l = 1.0f / l;
-  }
-  __syncthreads();
-  for (int i = tid; i < D; i += kCombineThreads) {
-    float a = 0.f;
-    for (int s = 0; s < S; ++s) a = fmaf(src[(long)s * (D + 2) + 2 + i], wgt[s], a);
-    o[i] = a * inv_l;
-  }
-#pragma unroll 1
-  for (int hh = 1; hh < D; hh <<= 1) {
-    __syncthreads();
-    for (int p = tid; p < D / 2; p += kCombineThreads) {
-      const int j = (p / hh) * 2 * hh + (p % hh);
-      const float a = o[j], c = o[j + hh];
-      o[j] = a + c;
-      o[j + hh] = a - c;
+      l = fmaf(ls[i], w, l);
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[1][warp] = l;
   __syncthreads();
-  const float inv_d = 1.0f / (float)D;
-  for (int i = tid; i < D; i += kCombineThreads) {
-    const float v = o[i] * inv_d;
-    dst[i] = ((tb.s1[i >> 5] >> (i & 31)) & 1u) ? -v : v;
+  l = red[1][0];
+#pragma unroll
+  for (int w = 1; w < W; ++w) l += red[1][w];
+  float a[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) a[e] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += W * PER) {
+    if (s0 > 0) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int s = s0 + warp + W * i;
+        if (s < S) {
+#pragma unroll
+          for (int v = 0; v < E / 4; ++v)
+            ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * D + lane * E)[v];
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int s = s0 + warp + W * i;
+      if (s < S) {
+        const float w = wgt[s];
+#pragma unroll
+        for (int v = 0; v < E / 4; ++v) {
+          a[4 * v] = fmaf(ov[i][v].x, w, a[4 * v]);
+          a[4 * v + 1] = fmaf(ov[i][v].y, w, a[4 * v + 1]);
+          a[4 * v + 2] = fmaf(ov[i][v].z, w, a[4 * v + 2]);
+          a[4 * v + 3] = fmaf(ov[i][v].w, w, a[4 * v + 3]);
+        }
+      }
+    }
   }
+#pragma unroll
+  for (int e = 0; e < E; ++e) part[warp][lane * E + e] = a[e];
+  __syncthreads();
+  if (warp == 0) {
+    const float inv = 1.0f / (l * (float)D);
+    float u[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int ch = lane * E + e;
+      float v = part[0][ch];
+#pragma unroll
+      for (int w = 1; w < W; ++w) v += part[w][ch];
+      u[e] = v;
+    }
+    warp_fwht<E>(u, lane);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int ch = lane * E + e;
+      const float v = u[e] * inv;
+      dst[ch] = ((tb.s1[ch >> 5] >> (ch & 31)) & 1u) ? -v : v;
+    }
+  }
+  pdl_trigger();
 }
 
 }  // namespace
@@ -108,13 +183,22 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
   else if (tb.d == 256)
     e = launch_decode_dim<256>(tb, cv, q, dtype, q_heads, scale_log2, plan, workspace, stream);
   if (e != cudaSuccess) return e;
-  dim3 grid(q_heads, cv.batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q_heads, cv.batch);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (tb.d == 128)
-    combine_kernel<128><<<grid, kCombineThreads, 0, stream>>>(tb, cv.seq_lens, cv.status, workspace,
-                                                             q_heads, plan.splits, plan.chunk, cv.capacity, out);
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<128>, tb, cv.seq_lens, cv.status,
+                           (const float*)workspace, q_heads, plan.splits, plan.chunk, cv.capacity, out);
   else
-    combine_kernel<256><<<grid, kCombineThreads, 0, stream>>>(tb, cv.seq_lens, cv.status, workspace,
-                                                             q_heads, plan.splits, plan.chunk, cv.capacity, out);
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<256>, tb, cv.seq_lens, cv.status,
+                           (const float*)workspace, q_heads, plan.splits, plan.chunk, cv.capacity, out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

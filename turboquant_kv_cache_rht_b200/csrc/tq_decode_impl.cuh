@@ -1,24 +1,37 @@
 // Fused decode attention on the packed TurboQuant cache (kernel template).
 //
 // One CTA handles one (split of the context, KV head, batch row) for all G
-// query heads that share the KV head ("How to Use TurboQuant ...", "What is
-// TurboQuant?": fused scoring kernels on packed low-bit data, GQA heads
+// query heads sharing that KV head ("How to Use TurboQuant ...", "What is
+// TurboQuant?": fused scoring kernels on packed low-bit data with query heads
 // repeated over a shared KV head; "TurboQuant Performance Benefits ...",
-// "Custom Metal Kernel Implementation": scores fused with value aggregation,
-// no dequantization pass).  Per 128-token tile:
-//   - cp.async stages the tile's key codes, value codes, norms (and QJL sign
-//     words and residual norms) into shared memory, one tile ahead;
-//   - key phase: thread t scores token t for the G heads directly on its code
-//     bits: sum_i q_rot[g][i] * c_K[code_i] through a shared-memory codebook,
-//     times the token's norm, plus the QJL sign-sketch term;
-//   - online softmax (running max / sum, base-2 exponent);
-//   - value phase: lane l accumulates channels l*d/32 .. for the G heads over
-//     the tile's tokens, again straight from the packed codes.
-// The rotated query and all constant factors (softmax scale, log2(e), the
-// 1/sqrt(d) of the rotation and of the dequantization, sqrt(pi/(2d)) of QJL)
-// are folded into the query once per CTA.  The partial (max, sum, output) of
-// each head goes to the workspace; a combine kernel merges the splits in a
-// fixed order and applies the inverse rotation.
+// "Custom Metal Kernel Implementation": scoring fused with value aggregation,
+// no dequantization pass; "mlx-turboquant" README, "The 1-bit QJL residual":
+// the sketch correction).
+//
+// For a GQA group the score and the aggregation are small dense contractions
+// (G rows of queries against a tile of tokens), so both run on the tensor
+// cores with mma.sync m16n8k16 (fp16 operands, fp32 accumulation):
+//   scores  S[token][col]  = K_hat[token][ch] . Qt[ch][col]
+//   output  O^T[ch][col]  += V_hat^T[ch][token] . P^T[token][col]
+// where a column is (head, part): the query and the probabilities are split
+// into fp16 hi + lo parts, so their products carry about 22 bits.  Key values
+// are split the same way (centroid = hi + lo, both fp16); value centroids are
+// used at fp16 precision.  The packed codes never become a dequantized
+// cache: each thread turns its own code bits into MMA fragment registers
+// through small pair tables (two codes -> two fp16 values) in shared memory.
+//
+// The MMA reduction order is free, so channels are assigned to fragment
+// slots such that every thread reads one contiguous slice of each packed row:
+//   keys  : thread quarter q owns channels [q*d/4, (q+1)*d/4) of tokens g, g+8
+//   values: thread group g owns channels [g*d/8, (g+1)*d/8) of tokens
+//           2q, 2q+1, 2q+8, 2q+9
+//   signs : like keys, pairing bits (j, j+16) of a word so one shift places
+//           both sign bits of a half2 (+-1.0 needs no table)
+// Tiles of 64 tokens (one 16-token slab per warp) are staged by cp.async in a
+// 3-stage pipeline.  Each warp keeps its own online-softmax state; the four
+// warps are merged in a fixed order and the CTA's partial (max, sum, output)
+// goes to the workspace, where the combine kernel merges the splits and
+// applies the inverse rotation.
 #pragma once
 
 #include "tq_internal.cuh"
@@ -28,8 +41,10 @@
 
 namespace tq {
 
-constexpr int kDecThreads = 128;
-constexpr int kDecTile = 128;  // tokens per tile: one per thread in the key phase
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecTile = 16 * kDecWarps;  // tokens per pipeline stage
+constexpr int kDecStages = 3;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -43,6 +58,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ float load_any(const void* p, long i, int dtype) {
   switch (dtype) {
     case kBF16: return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
@@ -51,61 +74,192 @@ __device__ __forceinline__ float load_any(const void* p, long i, int dtype) {
   }
 }
 
-template <int G>
-__device__ __forceinline__ void load_group(const float* p, float (&o)[G]) {
-  if constexpr (G % 4 == 0) {
-#pragma unroll
-    for (int g = 0; g < G; g += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(p + g);
-      o[g] = v.x; o[g + 1] = v.y; o[g + 2] = v.z; o[g + 3] = v.w;
-    }
-  } else if constexpr (G == 2) {
-    const float2 v = *reinterpret_cast<const float2*>(p);
-    o[0] = v.x; o[1] = v.y;
-  } else {
-    o[0] = p[0];
-  }
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-// code of channel i in a little-endian bit stream held in registers
-template <int B>
-__device__ __forceinline__ uint32_t code_at(const uint32_t* words, int i) {
-  const int off = B * i, w = off >> 5, s = off & 31;
-  if (s + B <= 32) return (words[w] >> s) & ((1u << B) - 1u);
-  return __funnelshift_r(words[w], words[w + 1], s) & ((1u << B) - 1u);
+// (x, part): the fp16 hi part of x, or the fp16 rounding of the remainder.
+__device__ __forceinline__ __half split_part(float x, int part) {
+  const __half hi = __float2half_rn(x);
+  return part ? __float2half_rn(x - __half2float(hi)) : hi;
+}
+
+// 2^x with the hardware approximation (relative error ~2^-22); x <= 0 here.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (a, b) -> half2 of their fp16 roundings (hi) and of the remainders (lo).
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Bits [off, off + width) of a little-endian stream held in registers w[0..n),
+// returned shifted left by `scale` (a byte offset into a table of 2^scale-byte
+// entries).  All arguments are compile-time constants after unrolling, so the
+// branches fold and w[] stays in registers.
+__device__ __forceinline__ uint32_t field_scaled(const uint32_t* w, int n, int off, int width,
+                                                 int scale) {
+  const uint32_t mask = ((1u << width) - 1u) << scale;
+  if (off < scale) return (w[0] << (scale - off)) & mask;
+  const int o = off - scale, wi = o >> 5, s = o & 31;
+  if (s == 0) return w[wi] & mask;
+  if (wi + 1 < n) return __funnelshift_r(w[wi], w[wi + 1], s) & mask;
+  return (w[wi] >> s) & mask;
+}
+
+// +-1.0 half2 from the two sign bits at positions 15 and 31 (bit 1 -> +1)
+__device__ __forceinline__ uint32_t sign_pair(uint32_t x) { return (x & 0x80008000u) ^ 0xBC00BC00u; }
+
+// Unnormalized Walsh-Hadamard transform of a d-vector spread over a warp
+// (lane l holds channels l*E .. l*E+E-1): in-lane butterflies, then shuffles.
+template <int E>
+__device__ __forceinline__ void warp_fwht(float (&u)[E], int lane) {
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+    for (int j = 0; j < E; ++j)
+      if ((j & h) == 0) {
+        const float a = u[j], c = u[j + h];
+        u[j] = a + c;
+        u[j + h] = a - c;
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float p = __shfl_xor_sync(0xffffffffu, u[e], m);
+      u[e] = (lane & m) ? p - u[e] : u[e] + p;
+    }
+}
+
+// Shared-memory row strides (32-bit words) of the staged codes, chosen so the
+// fragment loads below are free of bank conflicts (or as close as the access
+// pattern allows); multiples of 4 words for 16-byte copies.
+constexpr int k_stride_words(int d, int bits) { return (d == 256 && bits == 4) ? 36 : bits * d / 32; }
+constexpr int v_stride_words(int d, int bits) {
+  return d == 128 ? (bits == 4 ? 20 : 12) : (bits == 2 ? 20 : bits == 3 ? 28 : 36);
 }
 
 template <int D, int G, int KB, int VB, bool QJL>
 struct DecodeGeom {
-  static constexpr int kBytes = KB * D / 8;
-  static constexpr int vBytes = VB * D / 8;
-  static constexpr int sBytes = QJL ? D / 8 : 0;
-  static constexpr int kChunks = kBytes / 16;
-  static constexpr int vChunks = vBytes / 16;
-  static constexpr int sChunks = sBytes / 16;
-  // Odd row strides (in 16-byte chunks) keep the key phase's row-per-thread
-  // 128-bit reads free of bank conflicts.
-  static constexpr int kStride = (kChunks & 1) ? kChunks : kChunks + 1;
-  static constexpr int sStride = QJL ? ((sChunks & 1) ? sChunks : sChunks + 1) : 0;
+  static constexpr int NT = G > 4 ? 2 : 1;    // n-tiles of 8 columns (4 heads x {hi, lo})
+  static constexpr int KBLK = D / 16;         // 16-channel k-blocks of the score MMA
+  static constexpr int MBLK = D / 16;         // 16-channel m-blocks of the output MMA
+  static constexpr int kRowB = KB * D / 8;    // bytes of one packed row in global memory
+  static constexpr int vRowB = VB * D / 8;
+  static constexpr int sRowB = D / 8;
+  static constexpr int KS = k_stride_words(D, KB);
+  static constexpr int VS = v_stride_words(D, VB);
+  static constexpr int SS = D / 32;
+  static constexpr int KW = KB * D / 128;     // key words per thread quarter
+  static constexpr int SW = D / 128;          // sign words per thread quarter
+  static constexpr int VCH = VB * D / 8;      // value bits per thread group
+  static constexpr int VCW = (VCH + 31) / 32; // words of the aligned value chunk
+  static constexpr int VNW = (VCH % 32 == 0) ? VCH / 32 : (VCH + 16 + 31) / 32;
+  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (hi and lo half2 tables)
+  static constexpr int LV = 1 << (2 * VB);    // value pair-table entries (4 bytes each)
+  // Each table is replicated so that lanes with different (lane mod copies)
+  // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * size.
+  static constexpr int RKL = KB <= 3 ? 4 : 3;  // log2 key copies (16 or 8)
+  static constexpr int RVL = VB <= 3 ? 5 : 4;  // log2 value copies (32 or 16)
+  static constexpr int KSH = 2 + RKL;          // byte shift of a key entry index
+  static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
+  // one pipeline stage (bytes)
   static constexpr int offK = 0;
-  static constexpr int offV = offK + kDecTile * kStride * 16;
-  static constexpr int offS = offV + kDecTile * vChunks * 16 + 16;
-  static constexpr int offKN = offS + kDecTile * sStride * 16;
+  static constexpr int offV = offK + kDecTile * KS * 4;
+  static constexpr int offS = offV + kDecTile * VS * 4 + 16;
+  static constexpr int offKN = offS + (QJL ? kDecTile * SS * 4 : 0);
   static constexpr int offVN = offKN + kDecTile * 2;
   static constexpr int offRN = offVN + kDecTile * 2;
   static constexpr int stage = offRN + (QJL ? kDecTile * 2 : 0);
-  static constexpr int stageAligned = (stage + 127) / 128 * 128;
-  // shared-memory map after the two stages (bytes)
-  static constexpr int offQK = 2 * stageAligned;               // float [D][G]
-  static constexpr int offQQ = offQK + D * G * 4;               // float [D][G] (QJL)
-  static constexpr int offQB = offQQ + (QJL ? D * G * 4 : 0);   // float [G][D] scratch
-  static constexpr int offPW = offQB + D * G * 4;               // float [tile][G]
-  static constexpr int offLUT = offPW + kDecTile * G * 4;       // float [2][16]
-  static constexpr int offRED = offLUT + 32 * 4;                // float [4][G]
-  static constexpr int total = offRED + 4 * G * 4;
-  static_assert(4 * G * D * 4 <= 2 * stageAligned, "epilogue buffer must fit in the stages");
-  static_assert(VB * (D / 32) <= 32, "value chunk per lane must fit a word");
+  static constexpr int stageA = (stage + 127) / 128 * 128;
+  // epilogue merge buffer, reusing the stage area: per warp m[G], l[G], O[G][D]
+  static constexpr int mergeBytes = kDecWarps * G * (D + 2) * 4;
+  static constexpr int stagesBytes =
+      (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
+  // after the stage area
+  static constexpr int offLK = stagesBytes;
+  static constexpr int offLKlo = offLK + (LK << RKL) * 4;     // lo-part table after the hi-part one
+  static constexpr int offLV = offLK + (LK << RKL) * 8;
+  static constexpr int offQ = offLV + (LV << RVL) * 4;         // float [G][D] rotated query
+  static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
+  static constexpr int offRed = offQ2 + (QJL ? G * D * 4 : 0); // float [16]
+  static constexpr int total = offRed + 16 * 4;
+  static_assert((KS % 4) == 0 && (VS % 4) == 0, "16-byte aligned rows");
+  static_assert(VCW <= 4 && VNW <= 4, "value chunk too wide");
 };
+
+// Loads the value chunk of thread group g (bits [g*VCH, (g+1)*VCH)) of one
+// staged row into out[0..VCW), aligned to bit 0.
+template <int VCH, int VCW, int VNW>
+__device__ __forceinline__ void load_value_chunk(const uint32_t* row, int g, uint32_t (&out)[VCW]) {
+  const int bit = g * VCH, w0 = bit >> 5, sh = bit & 31;
+  uint32_t raw[VNW + 1];
+#pragma unroll
+  for (int i = 0; i < VNW; ++i) raw[i] = row[w0 + i];
+  raw[VNW] = 0u;
+  if constexpr (VCH % 32 == 0) {
+#pragma unroll
+    for (int i = 0; i < VCW; ++i) out[i] = raw[i];
+  } else {
+#pragma unroll
+    for (int i = 0; i < VCW; ++i) out[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
+  }
+}
+
+// x's bits [pos, pos + width), shifted to bit `scale` (either direction).
+__device__ __forceinline__ uint32_t bits_at(uint32_t x, int pos, int width, int scale) {
+  const uint32_t mask = ((1u << width) - 1u) << scale;
+  return pos >= scale ? (x >> (pos - scale)) & mask : (x << (scale - pos)) & mask;
+}
+
+// Interleaves the value chunks of two tokens a, b so that each 2*VB-bit field
+// holds (code_a | code_b << VB) of one channel: y for even channels, z for odd
+// ones (VB = 2 and 4; 3-bit codes are paired field by field instead).
+template <int VB, int VCW>
+__device__ __forceinline__ void interleave_pairs(const uint32_t (&a)[VCW], const uint32_t (&b)[VCW],
+                                                 uint32_t (&y)[VCW], uint32_t (&z)[VCW]) {
+#pragma unroll
+  for (int w = 0; w < VCW; ++w) {
+    if constexpr (VB == 4) {
+      y[w] = (a[w] & 0x0F0F0F0Fu) | ((b[w] & 0x0F0F0F0Fu) << 4);
+      z[w] = ((a[w] >> 4) & 0x0F0F0F0Fu) | (b[w] & 0xF0F0F0F0u);
+    } else if constexpr (VB == 2) {
+      y[w] = (a[w] & 0x33333333u) | ((b[w] & 0x33333333u) << 2);
+      z[w] = ((a[w] >> 2) & 0x33333333u) | (b[w] & 0xCCCCCCCCu);
+    } else {
+      y[w] = a[w];
+      z[w] = b[w];
+    }
+  }
+}
+
+// Byte offsets, into this lane's copy of the value pair table, of the pairs
+// (token a, token b) for channels 2mb (even) and 2mb + 1 (odd) of the chunk.
+template <int VB, int VCW, int VSH>
+__device__ __forceinline__ void value_pairs(const uint32_t (&y)[VCW], const uint32_t (&z)[VCW], int mb,
+                                            uint32_t lane_off, uint32_t& even, uint32_t& odd) {
+  if constexpr (VB == 4) {
+    const int w = mb >> 2, k = mb & 3;
+    even = bits_at(y[w], 8 * k, 8, VSH) | lane_off;
+    odd = bits_at(z[w], 8 * k, 8, VSH) | lane_off;
+  } else if constexpr (VB == 2) {
+    const int w = mb >> 3, k = mb & 7;
+    even = bits_at(y[w], 4 * k, 4, VSH) | lane_off;
+    odd = bits_at(z[w], 4 * k, 4, VSH) | lane_off;
+  } else {
+    const int o0 = VB * 2 * mb, o1 = o0 + VB;
+    even = field_scaled(y, VCW, o0, VB, VSH) | field_scaled(z, VCW, o0, VB, VSH + VB) | lane_off;
+    odd = field_scaled(y, VCW, o1, VB, VSH) | field_scaled(z, VCW, o1, VB, VSH + VB) | lane_off;
+  }
+}
 
 template <int D, int G, int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(kDecThreads)
@@ -113,265 +267,413 @@ __global__ void __launch_bounds__(kDecThreads)
                   const void* __restrict__ q, int q_dtype, int q_heads, float scale_log2,
                   int chunk, int splits, float* __restrict__ ws) {
   using Geo = DecodeGeom<D, G, KB, VB, QJL>;
-  constexpr int EV = D / 32;  // value channels per lane
+  constexpr int NT = Geo::NT;
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  pdl_wait();
   const int T = min(max(cv.seq_lens[b], 0), cv.capacity);  // never read past a row
   const int t_begin = split * chunk;
-  if (t_begin >= T) return;
+  if (t_begin >= T) {
+    pdl_trigger();
+    return;
+  }
   const int t_end = min(t_begin + chunk, T);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long row = (long)b * cv.kv_heads + kvh;
-  const long row_slot = row * cv.capacity;
+  const int g = lane >> 2, qd = lane & 3;
+  const long row_slot = ((long)b * cv.kv_heads + kvh) * cv.capacity;
 
-  float* qk = reinterpret_cast<float*>(smem + Geo::offQK);
-  float* qq = reinterpret_cast<float*>(smem + Geo::offQQ);
-  float* qb = reinterpret_cast<float*>(smem + Geo::offQB);
-  float* pw = reinterpret_cast<float*>(smem + Geo::offPW);
-  float* lutK = reinterpret_cast<float*>(smem + Geo::offLUT);
-  float* lutV = lutK + 16;
-  float* red = reinterpret_cast<float*>(smem + Geo::offRED);
-
+  // This thread's share of every tile copy: the chunk offsets are the same for
+  // all tiles, so they are computed once (stage offset and tile base vary).
+  constexpr int CK = Geo::kRowB / 16, CV = Geo::vRowB / 16, CS = Geo::sRowB / 16;
+  constexpr int NK = (kDecTile * CK + kDecThreads - 1) / kDecThreads;
+  constexpr int NV = (kDecTile * CV + kDecThreads - 1) / kDecThreads;
+  constexpr int NS = QJL ? (kDecTile * CS + kDecThreads - 1) / kDecThreads : 0;
+  int k_dst[NK], k_src[NK], k_row[NK], v_dst[NV], v_src[NV], v_row[NV];
+  int s_dst[NS > 0 ? NS : 1], s_row[NS > 0 ? NS : 1];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const int c = tid + kDecThreads * i, r = c / CK, col = c - r * CK;
+    k_row[i] = c < kDecTile * CK ? r : kDecTile;
+    k_dst[i] = Geo::offK + r * Geo::KS * 4 + col * 16;
+    k_src[i] = r * Geo::kRowB + col * 16;
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = tid + kDecThreads * i, r = c / CV, col = c - r * CV;
+    v_row[i] = c < kDecTile * CV ? r : kDecTile;
+    v_dst[i] = Geo::offV + r * Geo::VS * 4 + col * 16;
+    v_src[i] = r * Geo::vRowB + col * 16;
+  }
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    const int c = tid + kDecThreads * i;
+    s_row[i] = c < kDecTile * CS ? c / CS : kDecTile;
+    s_dst[i] = Geo::offS + c * 16;
+  }
   auto issue_tile = [&](int stage, int start) {
-    uint8_t* st = smem + stage * Geo::stageAligned;
+    uint8_t* st = smem + stage * Geo::stageA;
     const int n_valid = min(kDecTile, t_end - start);
     const int rows = (n_valid + 15) & ~15;  // within capacity (a multiple of 16)
-    const uint8_t* kc = cv.k_codes + (row_slot + start) * Geo::kBytes;
-    for (int c = tid; c < rows * Geo::kChunks; c += kDecThreads) {
-      const int r = c / Geo::kChunks, col = c - r * Geo::kChunks;
-      cp_async16(st + Geo::offK + (r * Geo::kStride + col) * 16, kc + r * Geo::kBytes + col * 16);
-    }
-    const uint8_t* vc = cv.v_codes + (row_slot + start) * Geo::vBytes;
-    for (int c = tid; c < rows * Geo::vChunks; c += kDecThreads)
-      cp_async16(st + Geo::offV + c * 16, vc + c * 16);
+    const uint8_t* kb = cv.k_codes + (row_slot + start) * Geo::kRowB;
+    const uint8_t* vb = cv.v_codes + (row_slot + start) * Geo::vRowB;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (k_row[i] < rows) cp_async16(st + k_dst[i], kb + k_src[i]);
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      if (v_row[i] < rows) cp_async16(st + v_dst[i], vb + v_src[i]);
     if constexpr (QJL) {
-      const uint8_t* sc = cv.k_signs + (row_slot + start) * Geo::sBytes;
-      for (int c = tid; c < rows * Geo::sChunks; c += kDecThreads) {
-        const int r = c / Geo::sChunks, col = c - r * Geo::sChunks;
-        cp_async16(st + Geo::offS + (r * Geo::sStride + col) * 16, sc + r * Geo::sBytes + col * 16);
-      }
+      const uint8_t* sb = cv.k_signs + (row_slot + start) * Geo::sRowB;
+#pragma unroll
+      for (int i = 0; i < NS; ++i)
+        if (s_row[i] < rows) cp_async16(st + s_dst[i], sb + (s_dst[i] - Geo::offS));
     }
-    const int nchunks = rows * 2 / 16;
-    for (int c = tid; c < nchunks; c += kDecThreads) {
-      cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
-      cp_async16(st + Geo::offVN + c * 16, reinterpret_cast<const uint8_t*>(cv.v_norm + row_slot + start) + c * 16);
-      if constexpr (QJL)
+    // norms: rows * 2 bytes each = rows / 8 chunks per array
+    const int c = tid & 7, arr = tid >> 3;
+    if (c < rows / 8) {
+      if (arr == 0)
+        cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
+      else if (arr == 1)
+        cp_async16(st + Geo::offVN + c * 16, reinterpret_cast<const uint8_t*>(cv.v_norm + row_slot + start) + c * 16);
+      else if (QJL && arr == 2)
         cp_async16(st + Geo::offRN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + c * 16);
     }
   };
 
+  const int n_tiles = (t_end - t_begin + kDecTile - 1) / kDecTile;
   issue_tile(0, t_begin);
   cp_async_commit();
+  if (n_tiles > 1) issue_tile(1, t_begin + kDecTile);
+  cp_async_commit();
 
-  // ---- rotate the G queries once: qk = H (s1 * q) * scale*log2(e)/d,
-  //      qq = H (s2 * H (s1 * q)) * scale*log2(e)*sqrt(pi/(2d))/d
-  if (tid < 16) {
-    lutK[tid] = tb.k_cent[tid];
-    lutV[tid] = tb.v_cent[tid];
+  // ---- pair tables: keys (hi pair, lo pair), values (fp16 pair)
+  {
+    // one thread per (entry, 16-byte group of copies): each group holds 4 copies
+    constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
+    for (int i = tid; i < Geo::LK * (RK / 4); i += kDecThreads) {
+      const int p = i / (RK / 4), grp = i % (RK / 4);
+      const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
+      const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
+      const __half la = __float2half_rn(ca - __half2float(ha));
+      const __half lb = __float2half_rn(cb - __half2float(hb));
+      const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
+      reinterpret_cast<uint4*>(smem + Geo::offLK)[p * (RK / 4) + grp] = make_uint4(hi, hi, hi, hi);
+      reinterpret_cast<uint4*>(smem + Geo::offLKlo)[p * (RK / 4) + grp] = make_uint4(lo, lo, lo, lo);
+    }
+    for (int i = tid; i < Geo::LV * (RV / 4); i += kDecThreads) {
+      const int p = i / (RV / 4), grp = i % (RV / 4);
+      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)]),
+                                    __float2half_rn(tb.v_cent[p >> VB]));
+      reinterpret_cast<uint4*>(smem + Geo::offLV)[p * (RV / 4) + grp] = make_uint4(v, v, v, v);
+    }
   }
+
+  // ---- rotate the G queries once, one warp per head, in registers:
+  //      u = H (s1 * q); QJL: w = H (s2 * u)
+  float* qs = reinterpret_cast<float*>(smem + Geo::offQ);
+  float* qs2 = reinterpret_cast<float*>(smem + Geo::offQ2);
+  float* red = reinterpret_cast<float*>(smem + Geo::offRed);
   const long q_base = ((long)b * q_heads + (long)kvh * G) * D;
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int ch = i % D;
-    const float x = load_any(q, q_base + i, q_dtype);
-    qb[i] = ((tb.s1[ch >> 5] >> (ch & 31)) & 1u) ? -x : x;
-  }
-  auto fwht_rows = [&]() {
-#pragma unroll 1
-    for (int h = 1; h < D; h <<= 1) {
-      __syncthreads();
-      for (int p = tid; p < G * D / 2; p += kDecThreads) {
-        const int g = p / (D / 2), k = p % (D / 2);
-        const int j = (k / h) * 2 * h + (k % h);
-        float* r = qb + g * D;
-        const float a = r[j], c = r[j + h];
-        r[j] = a + c;
-        r[j + h] = a - c;
+  float amax = 0.f, amax2 = 0.f;
+  for (int h = warp; h < G; h += kDecWarps) {
+    constexpr int E = D / 32;
+    float u[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int ch = lane * E + e;
+      const float x = load_any(q, q_base + (long)h * D + ch, q_dtype);
+      u[e] = ((tb.s1[ch >> 5] >> (ch & 31)) & 1u) ? -x : x;
+    }
+    warp_fwht<E>(u, lane);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      qs[h * D + lane * E + e] = u[e];
+      amax = fmaxf(amax, fabsf(u[e]));
+    }
+    if constexpr (QJL) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int ch = lane * E + e;
+        u[e] = ((tb.s2[ch >> 5] >> (ch & 31)) & 1u) ? -u[e] : u[e];
       }
-    }
-    __syncthreads();
-  };
-  fwht_rows();
-  const float ck = scale_log2 / (float)D;
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int g = i / D, ch = i % D;
-    qk[ch * G + g] = qb[i] * ck;
-  }
-  if constexpr (QJL) {
-    __syncthreads();
-    for (int i = tid; i < G * D; i += kDecThreads) {
-      const int ch = i % D;
-      if ((tb.s2[ch >> 5] >> (ch & 31)) & 1u) qb[i] = -qb[i];
-    }
-    fwht_rows();
-    const float cq = scale_log2 * sqrtf(3.14159265358979f / (2.0f * D)) / (float)D;
-    for (int i = tid; i < G * D; i += kDecThreads) {
-      const int g = i / D, ch = i % D;
-      qq[ch * G + g] = qb[i] * cq;
+      warp_fwht<E>(u, lane);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        qs2[h * D + lane * E + e] = u[e];
+        amax2 = fmaxf(amax2, fabsf(u[e]));
+      }
     }
   }
-
-  float m_run[G], l_part[G], acc[G][EV];
+  // power-of-two scales that bring each query table's largest entry just
+  // below 2^8, keeping the fp16 hi/lo parts in the normal range
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY;
-    l_part[g] = 0.f;
-#pragma unroll
-    for (int c = 0; c < EV; ++c) acc[g][c] = 0.f;
-  }
-
-  int it = 0;
-  for (int start = t_begin; start < t_end; start += kDecTile, ++it) {
-    const int stage = it & 1;
-    const bool has_next = start + kDecTile < t_end;
-    if (has_next) {
-      issue_tile(stage ^ 1, start + kDecTile);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint8_t* st = smem + stage * Geo::stageAligned;
-    const int n_valid = min(kDecTile, t_end - start);
-
-    // ---- key phase: thread tid scores token tid for the G heads
-    float s[G];
-    {
-      uint32_t kw[Geo::kChunks * 4];
-      const uint4* kr = reinterpret_cast<const uint4*>(st + Geo::offK + tid * Geo::kStride * 16);
-#pragma unroll
-      for (int c = 0; c < Geo::kChunks; ++c) {
-        const uint4 v = kr[c];
-        kw[4 * c] = v.x; kw[4 * c + 1] = v.y; kw[4 * c + 2] = v.z; kw[4 * c + 3] = v.w;
-      }
-      float ak[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) ak[g] = 0.f;
-#pragma unroll
-      for (int i = 0; i < D; ++i) {
-        const float val = lutK[code_at<KB>(kw, i)];
-        float qv[G];
-        load_group<G>(qk + i * G, qv);
-#pragma unroll
-        for (int g = 0; g < G; ++g) ak[g] = fmaf(qv[g], val, ak[g]);
-      }
-      const float kn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + Geo::offKN)[tid]));
-#pragma unroll
-      for (int g = 0; g < G; ++g) s[g] = ak[g] * kn;
-      if constexpr (QJL) {
-        uint32_t sw[Geo::sChunks * 4];
-        const uint4* sr = reinterpret_cast<const uint4*>(st + Geo::offS + tid * Geo::sStride * 16);
-#pragma unroll
-        for (int c = 0; c < Geo::sChunks; ++c) {
-          const uint4 v = sr[c];
-          sw[4 * c] = v.x; sw[4 * c + 1] = v.y; sw[4 * c + 2] = v.z; sw[4 * c + 3] = v.w;
-        }
-        float aq[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) aq[g] = 0.f;
-#pragma unroll
-        for (int i = 0; i < D; ++i) {
-          // bit 1 -> +q, bit 0 -> -q: flip the float sign bit when the code bit is 0
-          const uint32_t flip = ((~sw[i >> 5] >> (i & 31)) & 1u) << 31;
-          float qv[G];
-          load_group<G>(qq + i * G, qv);
-#pragma unroll
-          for (int g = 0; g < G; ++g) aq[g] += __uint_as_float(__float_as_uint(qv[g]) ^ flip);
-        }
-        const float rn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + Geo::offRN)[tid]));
-#pragma unroll
-        for (int g = 0; g < G; ++g) s[g] = fmaf(aq[g], rn, s[g]);
-      }
-      if (tid >= n_valid) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) s[g] = -INFINITY;
-      }
-    }
-
-    // ---- online softmax over the tile
-    float tmax[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float m = s[g];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      tmax[g] = m;
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) red[warp * G + g] = tmax[g];
-    }
-    __syncthreads();
-    const float vn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + Geo::offVN)[tid]));
-    float alpha[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float tm = fmaxf(fmaxf(red[g], red[G + g]), fmaxf(red[2 * G + g], red[3 * G + g]));
-      const float m_new = fmaxf(m_run[g], tm);
-      alpha[g] = exp2f(m_run[g] - m_new);
-      const float p = exp2f(s[g] - m_new);
-      l_part[g] = fmaf(l_part[g], alpha[g], p);
-      pw[tid * G + g] = (tid < n_valid) ? p * vn : 0.f;
-      m_run[g] = m_new;
-#pragma unroll
-      for (int c = 0; c < EV; ++c) acc[g][c] *= alpha[g];
-    }
-    __syncthreads();
-
-    // ---- value phase: warp w takes tokens w, w+4, ...; lane owns EV channels
-    {
-      constexpr int width = VB * EV;
-      const int off = lane * width, w0 = off >> 5, sh = off & 31;
-      const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Geo::offV);
-      for (int t = warp; t < n_valid; t += 4) {
-        const uint32_t* r = vrow + t * (Geo::vBytes / 4);
-        const uint32_t bits = __funnelshift_r(r[w0], r[w0 + 1], sh);
-        float pv[G];
-        load_group<G>(pw + t * G, pv);
-#pragma unroll
-        for (int c = 0; c < EV; ++c) {
-          const float val = lutV[(bits >> (VB * c)) & ((1u << VB) - 1u)];
-#pragma unroll
-          for (int g = 0; g < G; ++g) acc[g][c] = fmaf(pv[g], val, acc[g][c]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  // ---- epilogue: reduce the per-thread sums and the four warps' accumulators
-  float l_tot[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float l = l_part[g];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    l_tot[g] = l;
+  for (int o = 16; o > 0; o >>= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    amax2 = fmaxf(amax2, __shfl_xor_sync(0xffffffffu, amax2, o));
   }
   if (lane == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) red[warp * G + g] = l_tot[g];
+    red[warp] = amax;
+    red[8 + warp] = amax2;
   }
-  float* obuf = reinterpret_cast<float*>(smem);  // [4][G][D], the stages are free now
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int c = 0; c < EV; ++c) obuf[(warp * G + g) * D + lane * EV + c] = acc[g][c];
   __syncthreads();
-  float* dst = ws + ((long)(b * q_heads + kvh * G) * splits + split) * (D + 2);
-  const long head_stride = (long)splits * (D + 2);
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int g = i / D, ch = i % D;
-    const float o = ((obuf[(0 * G + g) * D + ch] + obuf[(1 * G + g) * D + ch]) +
-                     obuf[(2 * G + g) * D + ch]) + obuf[(3 * G + g) * D + ch];
-    dst[g * head_stride + 2 + ch] = o;
+  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  amax2 = fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
+  int e1 = 0, e2 = 0;
+  frexpf(amax > 0.f ? amax : 1.f, &e1);
+  frexpf(amax2 > 0.f ? amax2 : 1.f, &e2);
+  const float qsc = ldexpf(1.f, 8 - e1), qsc2 = ldexpf(1.f, 8 - e2);
+  // score = post * (tensor-core sum): undoes the query scale and folds the
+  // softmax scale, log2(e), the rotation's and the dequantization's 1/sqrt(d)
+  // (and sqrt(pi/(2d)) of the QJL estimate)
+  const float kpost = scale_log2 / ((float)D * qsc);
+  const float qpost = scale_log2 * sqrtf(3.14159265358979f / (2.0f * D)) / ((float)D * qsc2);
+
+  // ---- B fragments (query columns) in registers
+  uint32_t bk[NT][Geo::KBLK][2];
+  uint32_t bq[NT][QJL ? Geo::KBLK : 1][2];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 4 * j + (g >> 1), part = g & 1;
+    const bool live = head < G;
+    const float* r = qs + (live ? head : 0) * D;
+#pragma unroll
+    for (int kb = 0; kb < Geo::KBLK; ++kb) {
+      const int c0 = qd * (D / 4) + 4 * kb;  // key slots 2q,2q+1 -> c0,c0+1; 2q+8,2q+9 -> c0+2,c0+3
+      const uint32_t lo = pack_half2(split_part(r[c0] * qsc, part), split_part(r[c0 + 1] * qsc, part));
+      const uint32_t hi = pack_half2(split_part(r[c0 + 2] * qsc, part), split_part(r[c0 + 3] * qsc, part));
+      bk[j][kb][0] = live ? lo : 0u;
+      bk[j][kb][1] = live ? hi : 0u;
+      if constexpr (QJL) {
+        // sign slots 2q,2q+1 -> bits (j0, j0+16) of word kb/8; 2q+8,2q+9 -> (j0+8, j0+24)
+        const int base = qd * (D / 4) + 32 * (kb >> 3) + (kb & 7);
+        const float* r2 = qs2 + (live ? head : 0) * D;
+        const uint32_t s0 = pack_half2(split_part(r2[base] * qsc2, part), split_part(r2[base + 16] * qsc2, part));
+        const uint32_t s1 = pack_half2(split_part(r2[base + 8] * qsc2, part), split_part(r2[base + 24] * qsc2, part));
+        bq[j][kb][0] = live ? s0 : 0u;
+        bq[j][kb][1] = live ? s1 : 0u;
+      }
+    }
   }
-  if (tid < G) {
-    const int g = tid;
-    dst[g * head_stride + 0] = m_run[g];
-    dst[g * head_stride + 1] = ((red[g] + red[G + g]) + red[2 * G + g]) + red[3 * G + g];
+
+  // ---- per-warp online softmax state and output accumulators
+  float m_run[NT], l_part[NT];
+  float acc[NT][Geo::MBLK][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    m_run[j] = -INFINITY;
+    l_part[j] = 0.f;
+#pragma unroll
+    for (int mb = 0; mb < Geo::MBLK; ++mb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][mb][e] = 0.f;
   }
+  const uint8_t* lutK = smem + Geo::offLK;
+  const uint8_t* lutKlo = smem + Geo::offLKlo;
+  const uint8_t* lutV = smem + Geo::offLV;
+  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 2;
+  const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
+  const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
+
+  for (int it = 0; it < n_tiles; ++it) {
+    cp_async_wait<1>();
+    __syncthreads();
+    if (it + 2 < n_tiles) issue_tile((it + 2) % kDecStages, t_begin + (it + 2) * kDecTile);
+    cp_async_commit();
+
+    const uint8_t* st = smem + (it % kDecStages) * Geo::stageA;
+    const int n_valid = min(16, t_end - (t_begin + it * kDecTile + 16 * warp));
+    if (n_valid <= 0) continue;
+    const int r0 = 16 * warp;  // the warp's slab: rows r0 .. r0+15 of the stage
+
+    // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
+    float sacc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+    {
+      uint32_t kw0[Geo::KW], kw1[Geo::KW];
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS + qd * Geo::KW;
+#pragma unroll
+      for (int w = 0; w < Geo::KW; ++w) {
+        kw0[w] = k0[w];
+        kw1[w] = k0[8 * Geo::KS + w];
+      }
+#pragma unroll
+      for (int kb = 0; kb < Geo::KBLK; ++kb) {
+        const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
+        const uint32_t i0 = field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
+        const uint32_t i1 = field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
+        const uint32_t i2 = field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
+        const uint32_t i3 = field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
+        const uint32_t h0 = *reinterpret_cast<const uint32_t*>(lutK + i0);
+        const uint32_t h1 = *reinterpret_cast<const uint32_t*>(lutK + i1);
+        const uint32_t h2 = *reinterpret_cast<const uint32_t*>(lutK + i2);
+        const uint32_t h3 = *reinterpret_cast<const uint32_t*>(lutK + i3);
+        const uint32_t l0 = *reinterpret_cast<const uint32_t*>(lutKlo + i0);
+        const uint32_t l1 = *reinterpret_cast<const uint32_t*>(lutKlo + i1);
+        const uint32_t l2 = *reinterpret_cast<const uint32_t*>(lutKlo + i2);
+        const uint32_t l3 = *reinterpret_cast<const uint32_t*>(lutKlo + i3);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma16816(sacc[j], h0, h1, h2, h3, bk[j][kb][0], bk[j][kb][1]);
+          mma16816(sacc[j], l0, l1, l2, l3, bk[j][kb][0], bk[j][kb][1]);
+        }
+      }
+    }
+    const uint16_t* kn = reinterpret_cast<const uint16_t*>(st + Geo::offKN) + r0;
+    float s0[NT], s1[NT];
+    const float kn0 = __half2float(__ushort_as_half(kn[g])) * kpost;
+    const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      s0[j] = (sacc[j][0] + sacc[j][1]) * kn0;
+      s1[j] = (sacc[j][2] + sacc[j][3]) * kn1;
+    }
+    if constexpr (QJL) {
+      float qacc[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) qacc[j][0] = qacc[j][1] = qacc[j][2] = qacc[j][3] = 0.f;
+      uint32_t sw0[Geo::SW], sw1[Geo::SW];
+      const uint32_t* s0p = reinterpret_cast<const uint32_t*>(st + Geo::offS) + (r0 + g) * Geo::SS + qd * Geo::SW;
+#pragma unroll
+      for (int w = 0; w < Geo::SW; ++w) {
+        sw0[w] = s0p[w];
+        sw1[w] = s0p[8 * Geo::SS + w];
+      }
+#pragma unroll
+      for (int kb = 0; kb < Geo::KBLK; ++kb) {
+        const int wi = kb >> 3, j0 = kb & 7;
+        const uint32_t a0 = sign_pair(sw0[wi] << (15 - j0)), a1 = sign_pair(sw1[wi] << (15 - j0));
+        const uint32_t a2 = sign_pair(sw0[wi] << (7 - j0)), a3 = sign_pair(sw1[wi] << (7 - j0));
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(qacc[j], a0, a1, a2, a3, bq[j][kb][0], bq[j][kb][1]);
+      }
+      const uint16_t* rn = reinterpret_cast<const uint16_t*>(st + Geo::offRN) + r0;
+      const float rn0 = __half2float(__ushort_as_half(rn[g])) * qpost;
+      const float rn1 = __half2float(__ushort_as_half(rn[g + 8])) * qpost;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        s0[j] = fmaf(qacc[j][0] + qacc[j][1], rn0, s0[j]);
+        s1[j] = fmaf(qacc[j][2] + qacc[j][3], rn1, s1[j]);
+      }
+    }
+    const bool ok0 = g < n_valid, ok1 = g + 8 < n_valid;
+
+    // ---- online softmax (per warp, per head), P in fp16 hi/lo for the output MMA
+    const uint16_t* vn = reinterpret_cast<const uint16_t*>(st + Geo::offVN) + r0;
+    const float vn0 = __half2float(__ushort_as_half(vn[g]));
+    const float vn1 = __half2float(__ushort_as_half(vn[g + 8]));
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (!ok0) s0[j] = -INFINITY;
+      if (!ok1) s1[j] = -INFINITY;
+      float mx = fmaxf(s0[j], s1[j]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      if (mx > m_run[j]) {
+        const float alpha = fast_exp2(m_run[j] - mx);
+        l_part[j] *= alpha;
+#pragma unroll
+        for (int mb = 0; mb < Geo::MBLK; ++mb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[j][mb][e] *= alpha;
+        m_run[j] = mx;
+      }
+      const float p0 = ok0 ? fast_exp2(s0[j] - m_run[j]) : 0.f;
+      const float p1 = ok1 ? fast_exp2(s1[j] - m_run[j]) : 0.f;
+      l_part[j] += p0 + p1;
+      const float w0 = ok0 ? p0 * vn0 : 0.f, w1 = ok1 ? p1 * vn1 : 0.f;
+      uint32_t whi, wlo;
+      split_pair(w0, w1, whi, wlo);
+      const uint32_t x1h = __shfl_sync(0xffffffffu, whi, src1), x1l = __shfl_sync(0xffffffffu, wlo, src1);
+      const uint32_t x2h = __shfl_sync(0xffffffffu, whi, src2), x2l = __shfl_sync(0xffffffffu, wlo, src2);
+      const uint32_t x1 = (g & 1) ? x1l : x1h, x2 = (g & 1) ? x2l : x2h;
+      pb[j][0] = __byte_perm(x1, x2, 0x5410);  // tokens 2q, 2q+1
+      pb[j][1] = __byte_perm(x1, x2, 0x7632);  // tokens 2q+8, 2q+9
+    }
+
+    // ---- output: O^T += V_hat^T . P^T on the tensor cores
+    {
+      const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Geo::offV) + (r0 + 2 * qd) * Geo::VS;
+      uint32_t va[Geo::VCW], vb2[Geo::VCW], vc[Geo::VCW], vd[Geo::VCW];
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow, g, va);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + Geo::VS, g, vb2);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
+      uint32_t y0[Geo::VCW], z0[Geo::VCW], y1[Geo::VCW], z1[Geo::VCW];
+      interleave_pairs<VB, Geo::VCW>(va, vb2, y0, z0);
+      interleave_pairs<VB, Geo::VCW>(vc, vd, y1, z1);
+#pragma unroll
+      for (int mb = 0; mb < Geo::MBLK; ++mb) {
+        uint32_t e0, o0, e1, o1;
+        value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
+        value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j][mb], a0, a1, a2, a3, pb[j][0], pb[j][1]);
+      }
+    }
+  }
+
+  // ---- epilogue: merge the four warps (fixed order) into the CTA's partial
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    float l = l_part[j];
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    l_part[j] = l;
+  }
+  __syncthreads();  // every warp is done with the stages (no copies are in flight)
+  float* mw = reinterpret_cast<float*>(smem);  // [warp][G]
+  float* lw = mw + kDecWarps * G;              // [warp][G]
+  float* ow = lw + kDecWarps * G;              // [warp][G][D]
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 4 * j + qd;
+    if (head < G) {
+      if (g == 0) {
+        mw[warp * G + head] = m_run[j];
+        lw[warp * G + head] = l_part[j];
+      }
+      float* o = ow + (warp * G + head) * D + g * (D / 8);
+#pragma unroll
+      for (int mb = 0; mb < Geo::MBLK; ++mb) {
+        o[2 * mb] = acc[j][mb][0] + acc[j][mb][1];
+        o[2 * mb + 1] = acc[j][mb][2] + acc[j][mb][3];
+      }
+    }
+  }
+  __syncthreads();
+  // workspace: o partials [batch][q_heads][splits][D], then (m, l) [batch][q_heads][splits][2]
+  const long part0 = (long)(b * q_heads + kvh * G) * splits + split;
+  float* dst_o = ws + part0 * D;
+  float* dst_ml = ws + (long)gridDim.z * q_heads * splits * D + part0 * 2;
+  for (int i = tid; i < G * (D + 2); i += kDecThreads) {
+    const int h = i / (D + 2), e = i % (D + 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mw[w * G + h]);
+    float v = (e == 0) ? M : 0.f;
+    if (e > 0) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mwv = mw[w * G + h];
+        const float wt = (mwv == -INFINITY) ? 0.f : exp2f(mwv - M);
+        v = fmaf(e == 1 ? lw[w * G + h] : ow[(w * G + h) * D + (e - 2)], wt, v);
+      }
+    }
+    if (e < 2)
+      dst_ml[(long)h * splits * 2 + e] = v;
+    else
+      dst_o[(long)h * splits * D + (e - 2)] = v;
+  }
+  pdl_trigger();
 }
 
 // Launches decode_kernel for one compile-time shape (grid: splits x kv_heads x batch).
@@ -390,13 +692,21 @@ cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const voi
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  dim3 grid(plan.splits, cv.kv_heads, cv.batch);
-  kern<<<grid, kDecThreads, Geo::total, stream>>>(tb, cv, q, dtype, q_heads, scale_log2,
-                                                  plan.chunk, plan.splits, ws);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.splits, cv.kv_heads, cv.batch);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = Geo::total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tb, cv, q, dtype, q_heads, scale_log2, plan.chunk,
+                            plan.splits, ws);
 }
 
-// Per-head-dim dispatch over (group, k_bits, v_bits, qjl); defined in the
+// Per-head-dim dispatch over (group, k_bits, v_bits, qjl); instantiated in the
 // tq_decode_d<D>.cu translation units.
 template <int D>
 cudaError_t launch_decode_dim(const Tables& tb, const CacheView& cv, const void* q, int dtype,

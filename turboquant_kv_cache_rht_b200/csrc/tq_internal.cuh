@@ -8,6 +8,15 @@
 
 namespace tq {
 
+// Programmatic dependent launch.  Every kernel is launched with programmatic
+// stream serialization, waits for the previous kernel in the stream (and its
+// memory) before reading any buffer, and lets the next kernel start launching
+// once its own results are written.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 constexpr unsigned kFlagCapacity = 1u;  // mirrors TQ_FLAG_CAPACITY
 constexpr unsigned kFlagMaxCtx = 2u;    // mirrors TQ_FLAG_MAXCTX
 

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     s_bnd[1][tid] = tb.v_bnd[tid];
   }
   const int b = blockIdx.y;
+  pdl_wait();
   const int base = cv.seq_lens[b];
   const bool fits = base >= 0 && base <= cv.capacity - n_new;
   if (!fits && tid == 0 && blockIdx.x == 0) atomicOr(cv.status, (int)kFlagCapacity);
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       cv.append_sync[b] = 0;
     }
   }
+  pdl_trigger();
 }
 
 template <int D, typename T>
@@ -208,10 +210,17 @@ cudaError_t launch_typed(const Tables& tb, const CacheView& cv, const void* k, c
   const long vectors = 2L * cv.kv_heads * n_new;
   const long blocks = (vectors + kWarpsPerBlock - 1) / kWarpsPerBlock;
   if (blocks > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
-  dim3 grid((unsigned)blocks, (unsigned)cv.batch);
-  quantize_append_kernel<D, T><<<grid, kWarpsPerBlock * 32, 0, stream>>>(
-      tb, cv, static_cast<const T*>(k), static_cast<const T*>(v), n_new);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, (unsigned)cv.batch);
+  cfg.blockDim = dim3(kWarpsPerBlock * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_append_kernel<D, T>, tb, cv, static_cast<const T*>(k),
+                            static_cast<const T*>(v), n_new);
 }
 
 template <int D>
