@@ -165,6 +165,31 @@ tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, cons
                               tq_dtype dtype, int q_heads, float softmax_scale, int max_ctx,
                               float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode attention exactly like tq_decode_attention, for callers that cannot
+ * allocate device memory (and so cannot provide a workspace): for example a
+ * runtime whose device memory is reserved up front and managed by its own
+ * pool, a plugin that only receives input and output pointers from its host,
+ * or code that must not call cudaMalloc because an allocation can synchronize
+ * the device or fail at an unpredictable time.  The paper has no counterpart;
+ * this is a library-usability entry point.
+ *   - The per-split scratch lives in a static 8 MiB device array compiled into
+ *     the library; every GPU that loads the library holds it until the process
+ *     exits.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
+ *     library routine is called.
+ *   - A decode whose scratch (tq_decode_workspace_bytes for the same sizes)
+ *     exceeds 8 MiB is rejected with TQ_ERR_CAPACITY and enqueues nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (every partial is written before
+ *     it is read), but calls that overlap on the GPU (different streams, or
+ *     different threads without ordering) race on it: serialize them.
+ * Arguments, semantics and errors are otherwise those of tq_decode_attention. */
+tq_status tq_decode_attention_noalloc(const tq_codebook* cb, const tq_cache* cache, const void* q,
+                                      tq_dtype dtype, int q_heads, float softmax_scale,
+                                      int max_ctx, float* out, void* stream);
+
 /* Releases a codebook (NULL is ignored). */
 void tq_free(tq_codebook* cb);
 

@@ -178,6 +178,13 @@ tq_status cuda_status(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace tq {
+int record_error(int status, const char* message) {
+  g_last_error = message;
+  return status;
+}
+}  // namespace tq
+
 extern "C" {
 
 tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout* layout) {

@@ -59,4 +59,7 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
                           float* workspace, cudaStream_t stream);
 bool decode_supported(int head_dim, int group, int k_bits, int v_bits, int qjl);
 
+// Stores `message` as this thread's last error and returns `status`.
+int record_error(int status, const char* message);
+
 }  // namespace tq

@@ -28,7 +28,8 @@ TQ_FLAG_CAPACITY = 1
 TQ_FLAG_MAXCTX = 2
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append",
-           "tq_decode_workspace_bytes", "tq_decode_attention", "tq_free", "tq_last_error")
+           "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_noalloc",
+           "tq_free", "tq_last_error")
 
 
 class tq_params(C.Structure):
@@ -61,6 +62,9 @@ lib.tq_decode_attention.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p,
                                     C.c_float, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t,
                                     C.c_void_p]
 lib.tq_decode_attention.restype = C.c_int
+lib.tq_decode_attention_noalloc.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_int,
+                                            C.c_int, C.c_float, C.c_int, C.c_void_p, C.c_void_p]
+lib.tq_decode_attention_noalloc.restype = C.c_int
 lib.tq_free.argtypes = [C.c_void_p]
 lib.tq_free.restype = None
 lib.tq_last_error.argtypes = []
@@ -207,6 +211,28 @@ def tq_decode_attention(cb: Codebook, cache: Cache, q: torch.Tensor, out: torch.
                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                    _stream_ptr(stream)),
            "tq_decode_attention")
+    return out
+
+
+def tq_decode_attention_noalloc(cb: Codebook, cache: Cache, q: torch.Tensor,
+                                out: torch.Tensor | None = None, softmax_scale: float = 0.0,
+                                max_ctx: int | None = None, stream=None) -> torch.Tensor:
+    """tq_decode_attention without a workspace, for callers that cannot
+    allocate device memory: the library's built-in static scratch (8 MiB) is
+    used instead.  Calls share that scratch, so they must not overlap on the
+    GPU; make the first call on a device before any stream capture.  `out`
+    should be passed by such callers (allocating it here is only a
+    convenience)."""
+    if q.dim() != 3 or q.shape[0] != cache.batch or q.shape[2] != cb.head_dim or not q.is_contiguous():
+        raise ValueError("q must be contiguous [batch, q_heads, head_dim]")
+    max_ctx = cache.capacity if max_ctx is None else max_ctx
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    cs = cache.struct()
+    _check(lib.tq_decode_attention_noalloc(cb.handle, C.byref(cs), q.data_ptr(), _dtype_code(q),
+                                           q.shape[1], float(softmax_scale), int(max_ctx),
+                                           out.data_ptr(), _stream_ptr(stream)),
+           "tq_decode_attention_noalloc")
     return out
 
 
