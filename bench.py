@@ -139,6 +139,35 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def replica_plan(w: wl.Workload, steps_total: int, l2_bytes: int) -> dict:
+    """Cache replicas (total above 4x L2), appends per replica, capacity and
+    the decode's max_ctx for a run of `steps_total` appended steps."""
+    lengths = wl.context_lengths(w)
+    per_replica = sum(lengths) * w.kv_heads * token_bytes(w)
+    replicas = max(1, math.ceil(4 * l2_bytes / max(per_replica, 1)) + (0 if per_replica > 4 * l2_bytes else 1))
+    replicas = min(replicas, 64)
+    visits = math.ceil(steps_total / replicas) + 8
+    return {"lengths": lengths, "replicas": replicas,
+            "capacity": (max(lengths) + visits + 15) // 16 * 16, "max_ctx": max(lengths) + visits}
+
+
+def default_steps_total(steps: int = 200, warmup: int = 10) -> int:
+    """Appends one bench run makes per workload (timed + e2e steps + warm-up)."""
+    return 2 * steps + warmup
+
+
+def reduce_over_ranks(ms: float, byts: float, tokens: float, device) -> tuple[float, float, float]:
+    """Max of the device times and sums of the work over all ranks."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms, byts, tokens
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([byts, tokens], device=device, dtype=torch.float64)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u[0].item()), float(u[1].item())
+
+
 class State:
     """Caches (replicas), per-step inputs and outputs of one workload on one GPU."""
 
@@ -147,15 +176,12 @@ class State:
         self.tq = tq
         self.w = w
         self.dev = device
-        self.lengths = wl.context_lengths(w)
         self.cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed)
-        l2 = torch.cuda.get_device_properties(device).L2_cache_size
-        per_replica = sum(self.lengths) * w.kv_heads * token_bytes(w)
-        self.replicas = max(1, math.ceil(4 * l2 / max(per_replica, 1)) + (0 if per_replica > 4 * l2 else 1))
-        self.replicas = min(self.replicas, 64)
-        visits = math.ceil(steps_total / self.replicas) + 8
-        self.capacity = (max(self.lengths) + visits + 15) // 16 * 16
-        self.max_ctx = max(self.lengths) + visits
+        plan = replica_plan(w, steps_total, torch.cuda.get_device_properties(device).L2_cache_size)
+        self.lengths = plan["lengths"]
+        self.replicas = plan["replicas"]
+        self.capacity = plan["capacity"]
+        self.max_ctx = plan["max_ctx"]
         self.caches = [tq.Cache(self.cb, w.batch, w.kv_heads, self.capacity, device)
                        for _ in range(self.replicas)]
         self._prefill()
@@ -209,7 +235,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     dev = torch.device("cuda", local)
     w = wl.WORKLOADS[args.workload]
     K, W = args.steps, args.warmup
-    st = State(w, 2 * K + W, dev)
+    st = State(w, default_steps_total(K, W), dev)
     tq = st.tq
     stream = torch.cuda.current_stream(dev)
 
@@ -258,15 +284,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         lens = [L + grow for L in st.lengths]
         total_bytes += step_bytes(w, lens)["total"]
         ctx_tokens += sum(lens)
-    ms_max = ms
-    bytes_all, tokens_all = float(total_bytes), float(ctx_tokens)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        t = torch.tensor([bytes_all, tokens_all], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        bytes_all, tokens_all = float(t[0].item()), float(t[1].item())
+    ms_max, bytes_all, tokens_all = reduce_over_ranks(ms, float(total_bytes), float(ctx_tokens), dev)
 
     # ---- the decode call alone: events around each call, host queued ahead
     dec_ms = []

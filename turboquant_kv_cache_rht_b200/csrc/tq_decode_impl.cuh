@@ -163,13 +163,13 @@ struct DecodeGeom {
   static constexpr int VCH = VB * D / 8;      // value bits per thread group
   static constexpr int VCW = (VCH + 31) / 32; // words of the aligned value chunk
   static constexpr int VNW = (VCH % 32 == 0) ? VCH / 32 : (VCH + 16 + 31) / 32;
-  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (hi and lo half2 tables)
+  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (8 bytes: hi pair, lo pair)
   static constexpr int LV = 1 << (2 * VB);    // value pair-table entries (4 bytes each)
   // Each table is replicated so that lanes with different (lane mod copies)
   // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * size.
   static constexpr int RKL = KB <= 3 ? 4 : 3;  // log2 key copies (16 or 8)
   static constexpr int RVL = VB <= 3 ? 5 : 4;  // log2 value copies (32 or 16)
-  static constexpr int KSH = 2 + RKL;          // byte shift of a key entry index
+  static constexpr int KSH = 3 + RKL;          // byte shift of a key entry index (8-byte entries)
   static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
   // one pipeline stage (bytes)
   static constexpr int offK = 0;
@@ -186,12 +186,12 @@ struct DecodeGeom {
       (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
   // after the stage area
   static constexpr int offLK = stagesBytes;
-  static constexpr int offLKlo = offLK + (LK << RKL) * 4;     // lo-part table after the hi-part one
   static constexpr int offLV = offLK + (LK << RKL) * 8;
   static constexpr int offQ = offLV + (LV << RVL) * 4;         // float [G][D] rotated query
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
-  static constexpr int offRed = offQ2 + (QJL ? G * D * 4 : 0); // float [16]
-  static constexpr int total = offRed + 16 * 4;
+  static constexpr int offRed = offQ2 + (QJL ? G * D * 4 : 0); // float scratch
+  static constexpr int redFloats = (16 > 5 * G ? 16 : 5 * G) + 16;
+  static constexpr int total = offRed + redFloats * 4;
   static_assert((KS % 4) == 0 && (VS % 4) == 0, "16-byte aligned rows");
   static_assert(VCW <= 4 && VNW <= 4, "value chunk too wide");
 };
@@ -349,23 +349,24 @@ __global__ void __launch_bounds__(kDecThreads)
 
   // ---- pair tables: keys (hi pair, lo pair), values (fp16 pair)
   {
-    // one thread per (entry, 16-byte group of copies): each group holds 4 copies
+    // each entry is computed once and written to all its copies with 16-byte stores
     constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
-    for (int i = tid; i < Geo::LK * (RK / 4); i += kDecThreads) {
-      const int p = i / (RK / 4), grp = i % (RK / 4);
+    for (int p = tid; p < Geo::LK; p += kDecThreads) {
       const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
       const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
       const __half la = __float2half_rn(ca - __half2float(ha));
       const __half lb = __float2half_rn(cb - __half2float(hb));
       const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
-      reinterpret_cast<uint4*>(smem + Geo::offLK)[p * (RK / 4) + grp] = make_uint4(hi, hi, hi, hi);
-      reinterpret_cast<uint4*>(smem + Geo::offLKlo)[p * (RK / 4) + grp] = make_uint4(lo, lo, lo, lo);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 2);
+#pragma unroll
+      for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(hi, lo, hi, lo);
     }
-    for (int i = tid; i < Geo::LV * (RV / 4); i += kDecThreads) {
-      const int p = i / (RV / 4), grp = i % (RV / 4);
+    for (int p = tid; p < Geo::LV; p += kDecThreads) {
       const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)]),
                                     __float2half_rn(tb.v_cent[p >> VB]));
-      reinterpret_cast<uint4*>(smem + Geo::offLV)[p * (RV / 4) + grp] = make_uint4(v, v, v, v);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * (RV / 4);
+#pragma unroll
+      for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
     }
   }
 
@@ -440,18 +441,21 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
     for (int kb = 0; kb < Geo::KBLK; ++kb) {
       const int c0 = qd * (D / 4) + 4 * kb;  // key slots 2q,2q+1 -> c0,c0+1; 2q+8,2q+9 -> c0+2,c0+3
-      const uint32_t lo = pack_half2(split_part(r[c0] * qsc, part), split_part(r[c0 + 1] * qsc, part));
-      const uint32_t hi = pack_half2(split_part(r[c0 + 2] * qsc, part), split_part(r[c0 + 3] * qsc, part));
-      bk[j][kb][0] = live ? lo : 0u;
-      bk[j][kb][1] = live ? hi : 0u;
+      const float4 x = *reinterpret_cast<const float4*>(r + c0);
+      uint32_t h01, l01, h23, l23;
+      split_pair(x.x * qsc, x.y * qsc, h01, l01);
+      split_pair(x.z * qsc, x.w * qsc, h23, l23);
+      bk[j][kb][0] = live ? (part ? l01 : h01) : 0u;
+      bk[j][kb][1] = live ? (part ? l23 : h23) : 0u;
       if constexpr (QJL) {
         // sign slots 2q,2q+1 -> bits (j0, j0+16) of word kb/8; 2q+8,2q+9 -> (j0+8, j0+24)
         const int base = qd * (D / 4) + 32 * (kb >> 3) + (kb & 7);
         const float* r2 = qs2 + (live ? head : 0) * D;
-        const uint32_t s0 = pack_half2(split_part(r2[base] * qsc2, part), split_part(r2[base + 16] * qsc2, part));
-        const uint32_t s1 = pack_half2(split_part(r2[base + 8] * qsc2, part), split_part(r2[base + 24] * qsc2, part));
-        bq[j][kb][0] = live ? s0 : 0u;
-        bq[j][kb][1] = live ? s1 : 0u;
+        uint32_t a_h, a_l, b_h, b_l;
+        split_pair(r2[base] * qsc2, r2[base + 16] * qsc2, a_h, a_l);
+        split_pair(r2[base + 8] * qsc2, r2[base + 24] * qsc2, b_h, b_l);
+        bq[j][kb][0] = live ? (part ? a_l : a_h) : 0u;
+        bq[j][kb][1] = live ? (part ? b_l : b_h) : 0u;
       }
     }
   }
@@ -469,9 +473,8 @@ __global__ void __launch_bounds__(kDecThreads)
       for (int e = 0; e < 4; ++e) acc[j][mb][e] = 0.f;
   }
   const uint8_t* lutK = smem + Geo::offLK;
-  const uint8_t* lutKlo = smem + Geo::offLKlo;
   const uint8_t* lutV = smem + Geo::offLV;
-  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 2;
+  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 3;
   const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
   const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
 
@@ -487,9 +490,11 @@ __global__ void __launch_bounds__(kDecThreads)
     const int r0 = 16 * warp;  // the warp's slab: rows r0 .. r0+15 of the stage
 
     // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
-    float sacc[NT][4];
+    float sacc[NT][4], sacc2[NT][4];  // tokens g (hi/lo rows) and g + 8
 #pragma unroll
-    for (int j = 0; j < NT; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[j][e] = sacc2[j][e] = 0.f;
     {
       uint32_t kw0[Geo::KW], kw1[Geo::KW];
       const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS + qd * Geo::KW;
@@ -501,22 +506,15 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
-        const uint32_t i0 = field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
-        const uint32_t i1 = field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
-        const uint32_t i2 = field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
-        const uint32_t i3 = field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
-        const uint32_t h0 = *reinterpret_cast<const uint32_t*>(lutK + i0);
-        const uint32_t h1 = *reinterpret_cast<const uint32_t*>(lutK + i1);
-        const uint32_t h2 = *reinterpret_cast<const uint32_t*>(lutK + i2);
-        const uint32_t h3 = *reinterpret_cast<const uint32_t*>(lutK + i3);
-        const uint32_t l0 = *reinterpret_cast<const uint32_t*>(lutKlo + i0);
-        const uint32_t l1 = *reinterpret_cast<const uint32_t*>(lutKlo + i1);
-        const uint32_t l2 = *reinterpret_cast<const uint32_t*>(lutKlo + i2);
-        const uint32_t l3 = *reinterpret_cast<const uint32_t*>(lutKlo + i3);
+        // one MMA per 8 tokens: rows g / g+8 carry token g's hi / lo key parts
+        const uint2 p0 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint2 p1 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+        const uint2 p2 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          mma16816(sacc[j], h0, h1, h2, h3, bk[j][kb][0], bk[j][kb][1]);
-          mma16816(sacc[j], l0, l1, l2, l3, bk[j][kb][0], bk[j][kb][1]);
+          mma16816(sacc[j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
+          mma16816(sacc2[j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
         }
       }
     }
@@ -526,8 +524,8 @@ __global__ void __launch_bounds__(kDecThreads)
     const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      s0[j] = (sacc[j][0] + sacc[j][1]) * kn0;
-      s1[j] = (sacc[j][2] + sacc[j][3]) * kn1;
+      s0[j] = ((sacc[j][0] + sacc[j][1]) + (sacc[j][2] + sacc[j][3])) * kn0;
+      s1[j] = ((sacc2[j][0] + sacc2[j][1]) + (sacc2[j][2] + sacc2[j][3])) * kn1;
     }
     if constexpr (QJL) {
       float qacc[NT][4];
@@ -651,27 +649,33 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   __syncthreads();
   // workspace: o partials [batch][q_heads][splits][D], then (m, l) [batch][q_heads][splits][2]
+  float* wt = reinterpret_cast<float*>(smem + Geo::offRed);   // [warp][G] merge weights
+  if (tid < kDecWarps * G) {
+    const int w = tid / G, h = tid % G;
+    float M = mw[h];
+#pragma unroll
+    for (int v = 1; v < kDecWarps; ++v) M = fmaxf(M, mw[v * G + h]);
+    const float m = mw[w * G + h];
+    wt[tid] = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
+    if (w == 0) red[kDecWarps * G + h] = M;
+  }
+  __syncthreads();
   const long part0 = (long)(b * q_heads + kvh * G) * splits + split;
   float* dst_o = ws + part0 * D;
   float* dst_ml = ws + (long)gridDim.z * q_heads * splits * D + part0 * 2;
-  for (int i = tid; i < G * (D + 2); i += kDecThreads) {
-    const int h = i / (D + 2), e = i % (D + 2);
-    float M = -INFINITY;
+  for (int i = tid; i < G * D; i += kDecThreads) {
+    const int h = i / D, ch = i % D;
+    float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mw[w * G + h]);
-    float v = (e == 0) ? M : 0.f;
-    if (e > 0) {
+    for (int w = 0; w < kDecWarps; ++w) v = fmaf(ow[(w * G + h) * D + ch], wt[w * G + h], v);
+    dst_o[(long)h * splits * D + ch] = v;
+  }
+  if (tid < G) {
+    float l = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float mwv = mw[w * G + h];
-        const float wt = (mwv == -INFINITY) ? 0.f : exp2f(mwv - M);
-        v = fmaf(e == 1 ? lw[w * G + h] : ow[(w * G + h) * D + (e - 2)], wt, v);
-      }
-    }
-    if (e < 2)
-      dst_ml[(long)h * splits * 2 + e] = v;
-    else
-      dst_o[(long)h * splits * D + (e - 2)] = v;
+    for (int w = 0; w < kDecWarps; ++w) l = fmaf(lw[w * G + tid], wt[w * G + tid], l);
+    dst_ml[(long)tid * splits * 2] = red[kDecWarps * G + tid];
+    dst_ml[(long)tid * splits * 2 + 1] = l;
   }
   pdl_trigger();
 }
