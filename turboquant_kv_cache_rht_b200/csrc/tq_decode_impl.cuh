@@ -489,12 +489,27 @@ __global__ void __launch_bounds__(kDecThreads)
     if (n_valid <= 0) continue;
     const int r0 = 16 * warp;  // the warp's slab: rows r0 .. r0+15 of the stage
 
+    // value code chunks of tokens 2q, 2q+1, 2q+8, 2q+9, loaded early so their
+    // latency overlaps the score work
+    uint32_t va[Geo::VCW], vb2[Geo::VCW], vc[Geo::VCW], vd[Geo::VCW];
+    {
+      const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Geo::offV) + (r0 + 2 * qd) * Geo::VS;
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow, g, va);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + Geo::VS, g, vb2);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
+      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
+    }
+
     // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
-    float sacc[NT][4], sacc2[NT][4];  // tokens g (hi/lo rows) and g + 8
+    // tokens g (hi/lo rows) and g + 8, each split over even / odd k-blocks so
+    // that the MMA accumulation chains are half as long
+    float sacc[2][NT][4], sacc2[2][NT][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+    for (int par = 0; par < 2; ++par)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[j][e] = sacc2[j][e] = 0.f;
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[par][j][e] = sacc2[par][j][e] = 0.f;
     {
       uint32_t kw0[Geo::KW], kw1[Geo::KW];
       const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS + qd * Geo::KW;
@@ -513,8 +528,8 @@ __global__ void __launch_bounds__(kDecThreads)
         const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          mma16816(sacc[j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
-          mma16816(sacc2[j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
+          mma16816(sacc[kb & 1][j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
+          mma16816(sacc2[kb & 1][j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
         }
       }
     }
@@ -524,13 +539,17 @@ __global__ void __launch_bounds__(kDecThreads)
     const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      s0[j] = ((sacc[j][0] + sacc[j][1]) + (sacc[j][2] + sacc[j][3])) * kn0;
-      s1[j] = ((sacc2[j][0] + sacc2[j][1]) + (sacc2[j][2] + sacc2[j][3])) * kn1;
+      s0[j] = (((sacc[0][j][0] + sacc[1][j][0]) + (sacc[0][j][1] + sacc[1][j][1])) +
+               ((sacc[0][j][2] + sacc[1][j][2]) + (sacc[0][j][3] + sacc[1][j][3]))) * kn0;
+      s1[j] = (((sacc2[0][j][0] + sacc2[1][j][0]) + (sacc2[0][j][1] + sacc2[1][j][1])) +
+               ((sacc2[0][j][2] + sacc2[1][j][2]) + (sacc2[0][j][3] + sacc2[1][j][3]))) * kn1;
     }
     if constexpr (QJL) {
-      float qacc[NT][4];
+      float qacc[2][NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) qacc[j][0] = qacc[j][1] = qacc[j][2] = qacc[j][3] = 0.f;
+      for (int par = 0; par < 2; ++par)
+#pragma unroll
+        for (int j = 0; j < NT; ++j) qacc[par][j][0] = qacc[par][j][1] = qacc[par][j][2] = qacc[par][j][3] = 0.f;
       uint32_t sw0[Geo::SW], sw1[Geo::SW];
       const uint32_t* s0p = reinterpret_cast<const uint32_t*>(st + Geo::offS) + (r0 + g) * Geo::SS + qd * Geo::SW;
 #pragma unroll
@@ -544,15 +563,15 @@ __global__ void __launch_bounds__(kDecThreads)
         const uint32_t a0 = sign_pair(sw0[wi] << (15 - j0)), a1 = sign_pair(sw1[wi] << (15 - j0));
         const uint32_t a2 = sign_pair(sw0[wi] << (7 - j0)), a3 = sign_pair(sw1[wi] << (7 - j0));
 #pragma unroll
-        for (int j = 0; j < NT; ++j) mma16816(qacc[j], a0, a1, a2, a3, bq[j][kb][0], bq[j][kb][1]);
+        for (int j = 0; j < NT; ++j) mma16816(qacc[kb & 1][j], a0, a1, a2, a3, bq[j][kb][0], bq[j][kb][1]);
       }
       const uint16_t* rn = reinterpret_cast<const uint16_t*>(st + Geo::offRN) + r0;
       const float rn0 = __half2float(__ushort_as_half(rn[g])) * qpost;
       const float rn1 = __half2float(__ushort_as_half(rn[g + 8])) * qpost;
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        s0[j] = fmaf(qacc[j][0] + qacc[j][1], rn0, s0[j]);
-        s1[j] = fmaf(qacc[j][2] + qacc[j][3], rn1, s1[j]);
+        s0[j] = fmaf((qacc[0][j][0] + qacc[1][j][0]) + (qacc[0][j][1] + qacc[1][j][1]), rn0, s0[j]);
+        s1[j] = fmaf((qacc[0][j][2] + qacc[1][j][2]) + (qacc[0][j][3] + qacc[1][j][3]), rn1, s1[j]);
       }
     }
     const bool ok0 = g < n_valid, ok1 = g + 8 < n_valid;
@@ -594,12 +613,6 @@ __global__ void __launch_bounds__(kDecThreads)
 
     // ---- output: O^T += V_hat^T . P^T on the tensor cores
     {
-      const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Geo::offV) + (r0 + 2 * qd) * Geo::VS;
-      uint32_t va[Geo::VCW], vb2[Geo::VCW], vc[Geo::VCW], vd[Geo::VCW];
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow, g, va);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + Geo::VS, g, vb2);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
       uint32_t y0[Geo::VCW], z0[Geo::VCW], y1[Geo::VCW], z1[Geo::VCW];
       interleave_pairs<VB, Geo::VCW>(va, vb2, y0, z0);
       interleave_pairs<VB, Geo::VCW>(vc, vd, y1, z1);
