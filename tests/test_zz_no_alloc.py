@@ -57,12 +57,12 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_rejects_decodes_larger_than_its_scratch():
     cb = tq.Codebook(256, 2, 2, qjl=False, seed=0)
-    # 64 batch rows x 64 query heads at head_dim 256 need more than 8 MiB of partials
-    need = tq.tq_decode_workspace_bytes(cb, 64, 64, 8, 65536)
-    assert need > (8 << 20)
-    cache = tq.Cache(cb, 64, 8, 16, "cuda")
-    q = torch.zeros(64, 64, 256, dtype=torch.bfloat16, device="cuda")
-    out = torch.zeros(64, 64, 256, device="cuda")
+    # find a batch whose split partials need more than the 8 MiB static scratch
+    batch = next(bt for bt in (64, 128, 256, 512, 1024)
+                 if tq.tq_decode_workspace_bytes(cb, bt, 64, 8, 65536) > (8 << 20))
+    cache = tq.Cache(cb, batch, 8, 16, "cuda")
+    q = torch.zeros(batch, 64, 256, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(batch, 64, 256, device="cuda")
     cs = cache.struct()
     cs.capacity = 65536   # sizes only: the call is rejected before any launch
     st = tq.lib.tq_decode_attention_noalloc(cb.handle, C.byref(cs), q.data_ptr(), 1, 64, 0.0,
