@@ -46,6 +46,32 @@ METRIC = "fused TQ decode-attention GB/s & % HBM peak; ctx-tokens/s; quantize Mv
 FALLBACK_HBM_GBS = 6650.0
 
 
+# DRAM bytes (read + write) of one tq_decode_attention call (decode + combine
+# launches), per workload, from one ncu capture of `bench.py --workload <name>`
+# (dram__bytes_read.sum + dram__bytes_write.sum of both kernels).  Each entry
+# carries the digest of the decode sources it was taken with; once the kernel
+# sources change the figure no longer describes them and is reported as null.
+DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d128.cu", "tq_decode_d256.cu",
+                  "tq_internal.cuh")
+DECODE_TRAFFIC: dict[str, tuple[int, str]] = {}
+
+
+def decode_sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "turboquant_kv_cache_rht_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def decode_traffic(workload: str):
+    entry = DECODE_TRAFFIC.get(workload)
+    if entry is None or entry[1] != decode_sources_digest():
+        return None
+    return entry[0]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -347,7 +373,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "quantize_mvec_s": q_mvec,
         "roofline": {"bound": "hbm", "kernel": "tq_decode_attention (decode + combine launches)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(hbm_frac, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(hbm_frac, 4), "traffic": decode_traffic(w.name),
                      "algorithmic_bytes_per_launch": dec_bytes},
         "e2e": e2e,
         "gpu_launches": 3 * K,

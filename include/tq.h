@@ -140,7 +140,10 @@ tq_status tq_codebook_tables(const tq_codebook* cb, float* k_centroids, float* k
 tq_status tq_quantize_append(const tq_codebook* cb, const tq_cache* cache, const void* k,
                              const void* v, tq_dtype dtype, int n_new, void* stream);
 
-/* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes). */
+/* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes):
+ * (min(592, U * ceil(max_ctx / 64)) + U - 1) * (q_heads / kv_heads) *
+ * (head_dim + 2) * 4, U = batch * kv_heads -- one partial result per (CTA,
+ * unit) the decode's work partition can produce. */
 size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
                                  int max_ctx);
 
@@ -149,12 +152,16 @@ size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, 
  *       KV head h / (q_heads / kv_heads).
  * out : DEVICE float32 [batch][q_heads][head_dim].
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
- * max_ctx : host upper bound of every seq_lens[b] (at most capacity); it sizes
- *       the split over the context.  Tokens past it are not attended and set
- *       TQ_FLAG_MAXCTX.
+ * max_ctx : host upper bound of every seq_lens[b] (at most capacity); it
+ *       bounds the work partition and the workspace.  Tokens past it are not
+ *       attended and set TQ_FLAG_MAXCTX.  The partition itself is computed on
+ *       the device from seq_lens: every CTA takes an equal share of the token
+ *       tiles of all (batch row, KV head) pairs, so ragged batches stay
+ *       balanced.
  * workspace : DEVICE scratch of at least
  *       tq_decode_workspace_bytes(cb, batch, q_heads, kv_heads, max_ctx) bytes
- *       (TQ_ERR_CAPACITY otherwise); it holds the per-split partial results.
+ *       (TQ_ERR_CAPACITY otherwise); it holds the partial results.  Its
+ *       contents need no initialization.
  * Computes, for every (b, h), over tokens t < seq_lens[b]:
  *   s_t = scale * (<Rq, n_t c_K[code_t]/sqrt(d)>
  *                  + sqrt(pi/(2d)) * rho_t * <R2 R q, 2 bit_t - 1>)   (QJL term if enabled)

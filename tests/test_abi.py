@@ -116,13 +116,18 @@ def test_decode_validation():
 
 
 def test_workspace_size_formula():
+    # slots (one wave of at most 592 CTAs, no more CTAs than tiles, + units - 1)
+    # x group x (head_dim + 2) floats
+    def expect(batch, q_heads, kv_heads, max_ctx, d=128):
+        units = batch * kv_heads
+        ctas = max(1, min(148 * 4, units * max(1, -(-max_ctx // 64))))
+        return (ctas + units - 1) * (q_heads // kv_heads) * (d + 2) * 4
     cb = tq.Codebook(128, 3, 4)
-    ws = tq.tq_decode_workspace_bytes(cb, 1, 32, 8, 32768)
-    assert ws > 0 and ws % (130 * 4 * 32) == 0
-    splits = ws // (130 * 4 * 32)
-    assert 1 <= splits <= 512 and splits * 8 >= 148       # at least one wave of CTAs
-    assert tq.tq_decode_workspace_bytes(cb, 1, 30, 8, 100) == 0
-    assert tq.tq_decode_workspace_bytes(cb, 32, 32, 8, 65536) % (130 * 4 * 32 * 32) == 0
+    for args in ((1, 32, 8, 32768), (32, 32, 8, 65536), (1, 1, 1, 100), (1, 1, 1, 0), (4, 8, 8, 64)):
+        assert tq.tq_decode_workspace_bytes(cb, *args) == expect(*args), args
+    assert tq.tq_decode_workspace_bytes(cb, 1, 30, 8, 100) == 0              # group 3.75
+    cb256 = tq.Codebook(256, 2, 2)
+    assert tq.tq_decode_workspace_bytes(cb256, 2, 16, 4, 524288) == expect(2, 16, 4, 524288, 256)
 
 
 def test_kv_bits_split_matches_oracle():

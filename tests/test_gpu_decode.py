@@ -5,7 +5,7 @@ test_gpu_codec) and computes attention in float64; the GPU result must satisfy,
 for every (batch row, query head), max |gpu - oracle| <= 2e-3 * max |oracle|.
 Covers several tiles plus a ragged tail, lengths 0/1/127/128/129, all GQA
 groups, both head dims, every bit pair, QJL, custom softmax scale, repeat-run
-determinism, independence of the split count, and the max_ctx flag.
+determinism, independence of the work partition, and the max_ctx flag.
 """
 import numpy as np
 import pytest
@@ -103,7 +103,7 @@ def test_softmax_scale_and_fp32_query():
     assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
 
 
-def test_deterministic_and_split_independent():
+def test_deterministic_and_partition_independent():
     d, G, B, Hkv = 128, 2, 4, 8
     lengths = [3000, 2500, 1, 2999]
     cb, cache, k, v, q = _setup(d, 3, 4, True, B, Hkv, G, lengths, 8192, seed=8)
@@ -112,18 +112,47 @@ def test_deterministic_and_split_independent():
     b = tq.tq_decode_attention(cb, cache, qd, max_ctx=3000)
     torch.cuda.synchronize()
     assert torch.equal(a, b)                                  # bit-identical reruns
-    c = tq.tq_decode_attention(cb, cache, qd, max_ctx=8192)   # another split of the context
-    ws1 = tq.tq_decode_workspace_bytes(cb, B, Hkv * G, Hkv, 3000) // (B * Hkv * G * (d + 2) * 4)
-    ws2 = tq.tq_decode_workspace_bytes(cb, B, Hkv * G, Hkv, 8192) // (B * Hkv * G * (d + 2) * 4)
-    assert (3000 + ws1 - 1) // ws1 != (8192 + ws2 - 1) // ws2   # different chunk lengths
-    rel = ((a - c).abs().amax(-1) / a.abs().amax(-1)).max().item()
+    # the CTAs share out the tiles of all rows, so a longer row 2 moves every
+    # later CTA boundary: rows 0, 1 and 3 are then merged from other partials
+    cache.seq_lens[2] = 1700
+    c = tq.tq_decode_attention(cb, cache, qd, max_ctx=3000)
+    torch.cuda.synchronize()
+    cache.seq_lens[2] = 1
+    keep = [0, 1, 3]
+    rel = ((a[keep] - c[keep]).abs().amax(-1) / a[keep].abs().amax(-1)).max().item()
     assert rel <= 1e-5
+    assert not torch.equal(a[2], c[2])
     tb = oracle_tables(d, 3, 4, True, 8)
     for bb, h in ((0, 0), (3, 7), (2, 1)):
         n = lengths[bb]
         ek, ev = oracle_encode_unit(tb, k[bb, h, :n], v[bb, h, :n])
         ref = oracle_decode_unit(tb, q[bb, h * G:(h + 1) * G], ek, ev)
         assert_rows_close(a[bb, h * G:(h + 1) * G].cpu().numpy(), ref)
+    ek, ev = oracle_encode_unit(tb, k[2, 5, :1700], v[2, 5, :1700])    # row 2 at its new length
+    ref = oracle_decode_unit(tb, q[2, 5 * G:6 * G], ek, ev)
+    assert_rows_close(c[2, 5 * G:6 * G].cpu().numpy(), ref)
+
+
+def test_many_ragged_rows():
+    # 300 rows (more than one 128-row chunk of the decode's schedule and one
+    # 256-row pass of the combine's), a quarter of them empty, lengths 0..200:
+    # most CTAs meet several units and some rows end inside a CTA's range
+    d, G, B, Hkv = 128, 2, 300, 2
+    rng = np.random.default_rng(11)
+    lengths = [0 if rng.random() < 0.25 else int(rng.integers(1, 201)) for _ in range(B)]
+    cb, cache, k, v, q = _setup(d, 3, 4, False, B, Hkv, G, lengths, 208, seed=12)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=208).cpu()
+    torch.cuda.synchronize()
+    tb = oracle_tables(d, 3, 4, False, 12)
+    for bb in list(range(0, B, 7)) + [B - 1]:
+        for h in range(Hkv):
+            n = lengths[bb]
+            if n == 0:
+                assert torch.all(out[bb, h * G:(h + 1) * G] == 0)
+                continue
+            ek, ev = oracle_encode_unit(tb, k[bb, h, :n], v[bb, h, :n])
+            ref = oracle_decode_unit(tb, q[bb, h * G:(h + 1) * G], ek, ev)
+            assert_rows_close(out[bb, h * G:(h + 1) * G].numpy(), ref, what=f"row {bb} head {h}")
 
 
 def test_max_ctx_too_small_sets_flag():

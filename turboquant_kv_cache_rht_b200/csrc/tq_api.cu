@@ -260,8 +260,8 @@ size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, 
   if (!cb || batch <= 0 || q_heads <= 0 || kv_heads <= 0 || max_ctx < 0 ||
       q_heads % kv_heads != 0)
     return 0;
-  const tq::DecodePlan plan = tq::plan_decode(batch, kv_heads, max_ctx, cb->params.head_dim);
-  return tq::decode_workspace_bytes(plan, batch, q_heads, cb->params.head_dim);
+  const tq::DecodePlan plan = tq::plan_decode(batch, kv_heads, max_ctx, tq::kMaxTargetCtas);
+  return tq::decode_workspace_bytes(plan, q_heads, kv_heads, cb->params.head_dim);
 }
 
 tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, const void* q,
@@ -288,8 +288,8 @@ tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, cons
                 "no decode kernel for head_dim=%d group=%d k_bits=%d v_bits=%d qjl=%d "
                 "(group must be 1, 2, 4 or 8; v_bits must be k_bits or k_bits + 1)",
                 d, group, cb->params.k_bits, cb->params.v_bits, cb->params.qjl);
-  const tq::DecodePlan plan = tq::plan_decode(cache->batch, cache->kv_heads, max_ctx, d);
-  const size_t need = tq::decode_workspace_bytes(plan, cache->batch, q_heads, d);
+  const tq::DecodePlan plan = tq::plan_decode(cache->batch, cache->kv_heads, max_ctx, tq::kMaxTargetCtas);
+  const size_t need = tq::decode_workspace_bytes(plan, q_heads, cache->kv_heads, d);
   if (need > 0 && (!workspace || workspace_bytes < need))
     return fail(TQ_ERR_CAPACITY, "workspace of %zu bytes is smaller than the %zu needed",
                 workspace_bytes, need);
@@ -297,7 +297,7 @@ tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, cons
     return fail(TQ_ERR_INVALID, "workspace must be 16-byte aligned");
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
   return cuda_status(tq::launch_decode(cb->tables, view_of(cache), q, (int)dtype, q_heads, scale,
-                                       plan, out, (float*)workspace, (cudaStream_t)stream),
+                                       max_ctx, out, (float*)workspace, (cudaStream_t)stream),
                      "decode launch");
 }
 

@@ -8,65 +8,103 @@ namespace tq {
 namespace {
 
 constexpr int kCombineThreads = 256;
-constexpr int kMaxSplits = 512;
-// Split target: about four CTAs per SM of a 148-SM B200.  Fixed (not queried)
-// so that the workspace size is a pure function of the call's sizes.
-constexpr long kTargetCtas = 148L * 4;
+constexpr int kMaxParts = 1024;  // partials one unit can have (at most one per CTA)
+static_assert(kMaxTargetCtas <= kMaxParts, "a unit's partials must fit the merge");
 
-// Merges the splits of one (query head, batch row) and applies the inverse
-// rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
+// Merges the partial results of one (query head, batch row) and applies the
+// inverse rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
 // w_s = 2^(m_s - max m) ("How to Use TurboQuant ...", "What is TurboQuant?":
 // _rht_inverse; the 1/d collects the rotation's and the dequantization's
-// 1/sqrt(d)).  Every partial is loaded at once (warp w takes splits w, w+8,
-// ..., lane l channels l*d/32 ..), so the merge costs one memory round trip;
-// all reductions run in a fixed order.
+// 1/sqrt(d)).  The partials are those of the CTAs whose tile ranges meet the
+// unit's (the partition of DecodePlan, recomputed here from the lengths).
+// Every partial is loaded at once (warp w takes partials w, w+8, ..., lane l
+// channels l*d/32 ..), so the merge costs one memory round trip; all
+// reductions run in a fixed order.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const __grid_constant__ Tables tb, const int32_t* __restrict__ seq_lens,
-                   int32_t* status, const float* __restrict__ ws, int q_heads, int splits,
-                   int chunk, int capacity, float* __restrict__ out) {
+    combine_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
+                   const float* __restrict__ ws, int q_heads, int max_ctx, int nctas, int nslots,
+                   float* __restrict__ out) {
   constexpr int E = D / 32;
   constexpr int W = kCombineThreads / 32;
-  constexpr int PER = 8;  // splits per warp per round, loaded together
-  __shared__ float wgt[kMaxSplits];
+  constexpr int PER = 8;  // partials per warp per round, loaded together
+  __shared__ float wgt[kMaxParts];
   __shared__ __align__(16) float part[W][D];
   __shared__ float red[2][W];
+  __shared__ long long tiles_red[2][W];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = cv.kv_heads, G = q_heads / H, kvh = h / G, hg = h - kvh * G;
+  // The partition depends on the lengths alone, which the decode kernel does
+  // not write and which were complete before it let this grid launch: it is
+  // worked out before the wait, overlapping the decode's tail.
+  // tiles per KV head of the rows before b, and of all rows
+  long long before = 0, all = 0;
+  for (int r = tid; r < cv.batch; r += kCombineThreads) {
+    const long long x = row_tiles(cv, r, max_ctx);
+    all += x;
+    before += r < b ? x : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    all += __shfl_xor_sync(0xffffffffu, all, o);
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+  }
+  if (lane == 0) {
+    tiles_red[0][warp] = all;
+    tiles_red[1][warp] = before;
+  }
+  __syncthreads();
+  all = before = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    all += tiles_red[0][w];
+    before += tiles_red[1][w];
+  }
+  const int stored = min(max(cv.seq_lens[b], 0), cv.capacity);
+  const int n = row_tiles(cv, b, max_ctx);
+  float* dst = out + ((long)b * q_heads + h) * D;
+  // the CTAs c_lo .. c_hi whose ranges [c*T/nctas, (c+1)*T/nctas) meet [su, eu)
+  const long long T = all * H, su = before * H + (long long)kvh * n, eu = su + n;
+  const int c_lo = n > 0 ? (int)(((su + 1) * nctas + T - 1) / T - 1) : 0;
+  const int c_hi = n > 0 ? (int)((eu * nctas + T - 1) / T - 1) : -1;
+  const int S = c_hi - c_lo + 1;
   pdl_wait();
-  const long row = (long)b * q_heads + h;
-  const float* po = ws + row * splits * D;
-  const float* pml = ws + (long)gridDim.y * q_heads * splits * D + row * splits * 2;
+  if (tid == 0 && h == 0 && stored > max_ctx) atomicOr(cv.status, (int)kFlagMaxCtx);
+  if (n == 0) {
+    for (int i = tid; i < D; i += kCombineThreads) dst[i] = 0.f;
+    pdl_trigger();
+    return;
+  }
+
+  const long first = (long)c_lo + (long)b * H + kvh;  // slot of partial 0
+  const float* po = ws + (first * G + hg) * D;              // partial s at po + s * G * D
+  const float* pml = ws + (long)nslots * G * D + (first * G + hg) * 2;  // at pml + s * G * 2
   // issue the loads of the first round before anything depends on them
   float4 ov[PER][E / 4];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int s = warp + W * i;
-    if (s < splits) {
+    if (s < S) {
 #pragma unroll
       for (int v = 0; v < E / 4; ++v)
-        ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * D + lane * E)[v];
+        ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * G * D + lane * E)[v];
     }
   }
-  float ms[kMaxSplits / kCombineThreads], ls[kMaxSplits / kCombineThreads];
+  float ms[kMaxParts / kCombineThreads], ls[kMaxParts / kCombineThreads];
 #pragma unroll
-  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i) {
+  for (int i = 0; i < kMaxParts / kCombineThreads; ++i) {
     const int s = tid + kCombineThreads * i;
-    ms[i] = s < splits ? pml[2 * s] : -INFINITY;
-    ls[i] = s < splits ? pml[2 * s + 1] : 0.f;
-  }
-  const int T = min(max(seq_lens[b], 0), capacity);
-  if (tid == 0 && h == 0 && T > (long)splits * chunk) atomicOr(status, (int)kFlagMaxCtx);
-  const int S = min(splits, (T + chunk - 1) / chunk);
-  float* dst = out + row * D;
-  if (S <= 0) {
-    for (int i = tid; i < D; i += kCombineThreads) dst[i] = 0.f;
-    pdl_trigger();
-    return;
+    bool valid = false;
+    if (s < S) {  // a CTA with an empty range (T < nctas) left no partial
+      const long long c = c_lo + s, f0 = tile_bound(c, T, nctas), f1 = tile_bound(c + 1, T, nctas);
+      valid = max(f0, su) < min(f1, eu);
+    }
+    ms[i] = valid ? pml[(long)s * G * 2] : -INFINITY;
+    ls[i] = valid ? pml[(long)s * G * 2 + 1] : 0.f;
   }
   float m = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i)
-    if (tid + kCombineThreads * i < S) m = fmaxf(m, ms[i]);
+  for (int i = 0; i < kMaxParts / kCombineThreads; ++i) m = fmaxf(m, ms[i]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[0][warp] = m;
@@ -76,10 +114,10 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (int w = 1; w < W; ++w) m = fmaxf(m, red[0][w]);
   float l = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxSplits / kCombineThreads; ++i) {
+  for (int i = 0; i < kMaxParts / kCombineThreads; ++i) {
     const int s = tid + kCombineThreads * i;
     if (s < S) {
-      const float w = exp2f(ms[i] - m);
+      const float w = ms[i] == -INFINITY ? 0.f : exp2f(ms[i] - m);
       wgt[s] = w;
       l = fmaf(ls[i], w, l);
     }
@@ -102,7 +140,7 @@ __global__ void __launch_bounds__(kCombineThreads)
         if (s < S) {
 #pragma unroll
           for (int v = 0; v < E / 4; ++v)
-            ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * D + lane * E)[v];
+            ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * G * D + lane * E)[v];
         }
       }
     }
@@ -111,12 +149,14 @@ __global__ void __launch_bounds__(kCombineThreads)
       const int s = s0 + warp + W * i;
       if (s < S) {
         const float w = wgt[s];
+        if (w > 0.f) {  // skips the slots no CTA wrote
 #pragma unroll
-        for (int v = 0; v < E / 4; ++v) {
-          a[4 * v] = fmaf(ov[i][v].x, w, a[4 * v]);
-          a[4 * v + 1] = fmaf(ov[i][v].y, w, a[4 * v + 1]);
-          a[4 * v + 2] = fmaf(ov[i][v].z, w, a[4 * v + 2]);
-          a[4 * v + 3] = fmaf(ov[i][v].w, w, a[4 * v + 3]);
+          for (int v = 0; v < E / 4; ++v) {
+            a[4 * v] = fmaf(ov[i][v].x, w, a[4 * v]);
+            a[4 * v + 1] = fmaf(ov[i][v].y, w, a[4 * v + 1]);
+            a[4 * v + 2] = fmaf(ov[i][v].z, w, a[4 * v + 2]);
+            a[4 * v + 3] = fmaf(ov[i][v].w, w, a[4 * v + 3]);
+          }
         }
       }
     }
@@ -148,21 +188,17 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 }  // namespace
 
-DecodePlan plan_decode(int batch, int kv_heads, int max_ctx, int head_dim) {
-  (void)head_dim;
+DecodePlan plan_decode(int batch, int kv_heads, int max_ctx, long target_ctas) {
   const long tiles = std::max<long>(1, (max_ctx + kDecTile - 1) / kDecTile);
   const long units = std::max<long>(1, (long)batch * kv_heads);
-  long s = (kTargetCtas + units - 1) / units;
-  s = std::max<long>(1, std::min<long>({s, tiles, (long)kMaxSplits}));
-  const long per = (tiles + s - 1) / s;
   DecodePlan p;
-  p.splits = (int)((tiles + per - 1) / per);
-  p.chunk = (int)(per * kDecTile);
+  p.ctas = (int)std::max<long>(1, std::min(target_ctas, units * tiles));
+  p.slots = (int)(p.ctas + units - 1);
   return p;
 }
 
-size_t decode_workspace_bytes(const DecodePlan& plan, int batch, int q_heads, int head_dim) {
-  return (size_t)batch * q_heads * plan.splits * (head_dim + 2) * sizeof(float);
+size_t decode_workspace_bytes(const DecodePlan& plan, int q_heads, int kv_heads, int head_dim) {
+  return (size_t)plan.slots * (q_heads / kv_heads) * (head_dim + 2) * sizeof(float);
 }
 
 bool decode_supported(int head_dim, int group, int k_bits, int v_bits, int qjl) {
@@ -174,14 +210,27 @@ bool decode_supported(int head_dim, int group, int k_bits, int v_bits, int qjl) 
 }
 
 cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, int dtype,
-                          int q_heads, float scale, const DecodePlan& plan, float* out,
-                          float* workspace, cudaStream_t stream) {
+                          int q_heads, float scale, int max_ctx, float* out, float* workspace,
+                          cudaStream_t stream) {
   const float scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = cudaErrorNotSupported;
+  const int group = q_heads / cv.kv_heads;
+  // one wave of CTAs at the kernel's occupancy (capped at the workspace bound)
+  int ctas_per_sm = 0, sms = 0, dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = tb.d == 128 ? decode_occupancy_dim<128>(tb, group, &ctas_per_sm)
+                  : decode_occupancy_dim<256>(tb, group, &ctas_per_sm);
+  if (e != cudaSuccess) return e;
+  const long target = std::min<long>(kMaxTargetCtas, (long)std::max(ctas_per_sm, 1) * sms);
+  const DecodePlan plan = plan_decode(cv.batch, cv.kv_heads, max_ctx, target);
   if (tb.d == 128)
-    e = launch_decode_dim<128>(tb, cv, q, dtype, q_heads, scale_log2, plan, workspace, stream);
+    e = launch_decode_dim<128>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
   else if (tb.d == 256)
-    e = launch_decode_dim<256>(tb, cv, q, dtype, q_heads, scale_log2, plan, workspace, stream);
+    e = launch_decode_dim<256>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+  else
+    e = cudaErrorNotSupported;
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(q_heads, cv.batch);
@@ -193,11 +242,11 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (tb.d == 128)
-    e = cudaLaunchKernelEx(&cfg, combine_kernel<128>, tb, cv.seq_lens, cv.status,
-                           (const float*)workspace, q_heads, plan.splits, plan.chunk, cv.capacity, out);
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<128>, tb, cv, (const float*)workspace, q_heads,
+                           max_ctx, plan.ctas, plan.slots, out);
   else
-    e = cudaLaunchKernelEx(&cfg, combine_kernel<256>, tb, cv.seq_lens, cv.status,
-                           (const float*)workspace, q_heads, plan.splits, plan.chunk, cv.capacity, out);
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<256>, tb, cv, (const float*)workspace, q_heads,
+                           max_ctx, plan.ctas, plan.slots, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -1,7 +1,10 @@
 // Fused decode attention on the packed TurboQuant cache (kernel template).
 //
-// One CTA handles one (split of the context, KV head, batch row) for all G
-// query heads sharing that KV head ("How to Use TurboQuant ...", "What is
+// The grid is one wave of CTAs.  The token tiles of all (batch row, KV head)
+// units are laid end to end and every CTA takes an equal share of them, read
+// from the lengths on the device, so ragged batches stay balanced; each unit
+// a CTA meets (a segment) is processed for all G query heads sharing that KV
+// head ("How to Use TurboQuant ...", "What is
 // TurboQuant?": fused scoring kernels on packed low-bit data with query heads
 // repeated over a shared KV head; "TurboQuant Performance Benefits ...",
 // "Custom Metal Kernel Implementation": scoring fused with value aggregation,
@@ -29,9 +32,9 @@
 //           both sign bits of a half2 (+-1.0 needs no table)
 // Tiles of 64 tokens (one 16-token slab per warp) are staged by cp.async in a
 // 3-stage pipeline.  Each warp keeps its own online-softmax state; the four
-// warps are merged in a fixed order and the CTA's partial (max, sum, output)
-// goes to the workspace, where the combine kernel merges the splits and
-// applies the inverse rotation.
+// warps are merged in a fixed order and each segment's partial (max, sum,
+// output) goes to the workspace, where the combine kernel merges the
+// partials of every unit and applies the inverse rotation.
 #pragma once
 
 #include "tq_internal.cuh"
@@ -191,7 +194,11 @@ struct DecodeGeom {
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offRed = offQ2 + (QJL ? G * D * 4 : 0); // float scratch
   static constexpr int redFloats = (16 > 5 * G ? 16 : 5 * G) + 16;
-  static constexpr int total = offRed + redFloats * 4;
+  // work schedule: scan scratch (one 64-bit word per warp), then one chunk of
+  // rows (index, 64-bit tile prefix)
+  static constexpr int offSched = (offRed + redFloats * 4 + 15) / 16 * 16;
+  static constexpr int schedBytes = kDecWarps * 8 + kDecThreads * 4 + kDecThreads * 8;
+  static constexpr int total = offSched + schedBytes;
   static_assert((KS % 4) == 0 && (VS % 4) == 0, "16-byte aligned rows");
   static_assert(VCW <= 4 && VNW <= 4, "value chunk too wide");
 };
@@ -261,27 +268,124 @@ __device__ __forceinline__ void value_pairs(const uint32_t (&y)[VCW], const uint
   }
 }
 
+// Tokens of row b a decode call attends: seq_lens[b] clamped to the row's
+// capacity and to the call's max_ctx.
+__device__ __forceinline__ int row_len(const CacheView& cv, int b, int max_ctx) {
+  return min(min(max(cv.seq_lens[b], 0), cv.capacity), max_ctx);
+}
+__device__ __forceinline__ int row_tiles(const CacheView& cv, int b, int max_ctx) {
+  return (row_len(cv, b, max_ctx) + kDecTile - 1) / kDecTile;
+}
+
+// floor(c * T / n), the first tile of CTA c of n over T tiles (32-bit
+// division when the product fits, as it does for all but huge contexts).
+__device__ __forceinline__ long long tile_bound(long long c, long long T, int n) {
+  const long long num = c * T;
+  return num < (1ll << 32) ? (long long)((unsigned)num / (unsigned)n) : num / n;
+}
+
+// Block-wide exclusive prefix sum of one value per thread (NT threads, all of
+// them calling); *total receives the block's sum.  `scratch` holds NT/32
+// words of shared memory and is free again when the call returns.
+template <int NT>
+__device__ __forceinline__ long long block_exclusive_scan(long long x, long long* scratch,
+                                                          long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  long long before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const long long v = scratch[w];
+    before += w < warp ? v : 0;
+    all += v;
+  }
+  __syncthreads();
+  *total = all;
+  return before + inc - x;
+}
+
+// CTAs per SM the register budget is sized for: d = 128 fits four CTAs (128
+// registers) unless the shape carries two column tiles or the QJL sketch,
+// which need up to 168 registers (three CTAs); d = 256 fits two.
+template <int D, int G, bool QJL>
+constexpr int decode_min_ctas() { return D == 128 ? ((G > 4 || QJL) ? 3 : 4) : 2; }
+
 template <int D, int G, int KB, int VB, bool QJL>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     decode_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                   const void* __restrict__ q, int q_dtype, int q_heads, float scale_log2,
-                  int chunk, int splits, float* __restrict__ ws) {
+                  int max_ctx, int nslots, float* __restrict__ ws) {
   using Geo = DecodeGeom<D, G, KB, VB, QJL>;
   constexpr int NT = Geo::NT;
   extern __shared__ __align__(128) uint8_t smem[];
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  pdl_wait();
-  const int T = min(max(cv.seq_lens[b], 0), cv.capacity);  // never read past a row
-  const int t_begin = split * chunk;
-  if (t_begin >= T) {
-    pdl_trigger();
-    return;
-  }
-  const int t_end = min(t_begin + chunk, T);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, qd = lane & 3;
-  const long row_slot = ((long)b * cv.kv_heads + kvh) * cv.capacity;
+  const int H = cv.kv_heads;
+  // ---- pair tables: keys (hi pair, lo pair), values (fp16 pair).  They
+  //      depend on the kernel parameters alone, so they are built before the
+  //      wait, overlapping the previous kernel in the stream.
+  {
+    // each entry is computed once and written to all its copies with 16-byte stores
+    constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
+    for (int p = tid; p < Geo::LK; p += kDecThreads) {
+      const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
+      const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
+      const __half la = __float2half_rn(ca - __half2float(ha));
+      const __half lb = __float2half_rn(cb - __half2float(hb));
+      const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 2);
+#pragma unroll
+      for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(hi, lo, hi, lo);
+    }
+    for (int p = tid; p < Geo::LV; p += kDecThreads) {
+      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)]),
+                                    __float2half_rn(tb.v_cent[p >> VB]));
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * (RV / 4);
+#pragma unroll
+      for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
+    }
+  }
+
+  pdl_wait();
+
+  // ---- this CTA's tiles [t0, t1) of the T laid end to end over all units
+  long long* scan = reinterpret_cast<long long*>(smem + Geo::offSched);
+  int* row_n = reinterpret_cast<int*>(scan + kDecWarps);                      // [chunk row] tiles
+  long long* row_p = reinterpret_cast<long long*>(row_n + kDecThreads);      // [chunk row] prefix
+  // one chunk of rows (the usual case): the scan gives the prefixes and the
+  // total at once; otherwise a first pass sums the tiles of every chunk
+  const bool one_chunk = cv.batch <= kDecThreads;
+  long long rows_total = 0, x0 = 0, p0 = 0;
+  if (one_chunk) {
+    x0 = tid < cv.batch ? row_tiles(cv, tid, max_ctx) : 0;
+    p0 = block_exclusive_scan<kDecThreads>(x0, scan, &rows_total);
+  } else {
+    for (int b0 = 0; b0 < cv.batch; b0 += kDecThreads) {
+      const int r = b0 + tid;
+      long long tot;
+      block_exclusive_scan<kDecThreads>(r < cv.batch ? row_tiles(cv, r, max_ctx) : 0, scan, &tot);
+      rows_total += tot;
+    }
+  }
+  const long long T = rows_total * H;
+  const long long t0 = tile_bound(blockIdx.x, T, gridDim.x);
+  const long long t1 = tile_bound((long long)blockIdx.x + 1, T, gridDim.x);
+  // Everything the next kernel may read before its own wait (the lengths)
+  // was complete before this kernel's wait returned, so it may start now; it
+  // waits for this grid's completion before it reads any partial.
+  pdl_trigger();
+  if (t0 >= t1) return;
+  // the current segment: tokens [t_begin, t_end) of row b, KV head kvh
+  int b = 0, kvh = 0, t_begin = 0, t_end = 0;
+  long row_slot = 0;
 
   // This thread's share of every tile copy: the chunk offsets are the same for
   // all tiles, so they are computed once (stage offset and tile base vary).
@@ -341,34 +445,12 @@ __global__ void __launch_bounds__(kDecThreads)
     }
   };
 
+  auto segment = [&]() {
   const int n_tiles = (t_end - t_begin + kDecTile - 1) / kDecTile;
   issue_tile(0, t_begin);
   cp_async_commit();
   if (n_tiles > 1) issue_tile(1, t_begin + kDecTile);
   cp_async_commit();
-
-  // ---- pair tables: keys (hi pair, lo pair), values (fp16 pair)
-  {
-    // each entry is computed once and written to all its copies with 16-byte stores
-    constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
-    for (int p = tid; p < Geo::LK; p += kDecThreads) {
-      const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
-      const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
-      const __half la = __float2half_rn(ca - __half2float(ha));
-      const __half lb = __float2half_rn(cb - __half2float(hb));
-      const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 2);
-#pragma unroll
-      for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(hi, lo, hi, lo);
-    }
-    for (int p = tid; p < Geo::LV; p += kDecThreads) {
-      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)]),
-                                    __float2half_rn(tb.v_cent[p >> VB]));
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * (RV / 4);
-#pragma unroll
-      for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
-    }
-  }
 
   // ---- rotate the G queries once, one warp per head, in registers:
   //      u = H (s1 * q); QJL: w = H (s2 * u)
@@ -661,7 +743,7 @@ __global__ void __launch_bounds__(kDecThreads)
     }
   }
   __syncthreads();
-  // workspace: o partials [batch][q_heads][splits][D], then (m, l) [batch][q_heads][splits][2]
+  // workspace: o partials [slot][G][D], then (m, l) [slot][G][2]; slot = CTA + unit
   float* wt = reinterpret_cast<float*>(smem + Geo::offRed);   // [warp][G] merge weights
   if (tid < kDecWarps * G) {
     const int w = tid / G, h = tid % G;
@@ -673,44 +755,99 @@ __global__ void __launch_bounds__(kDecThreads)
     if (w == 0) red[kDecWarps * G + h] = M;
   }
   __syncthreads();
-  const long part0 = (long)(b * q_heads + kvh * G) * splits + split;
-  float* dst_o = ws + part0 * D;
-  float* dst_ml = ws + (long)gridDim.z * q_heads * splits * D + part0 * 2;
+  const long slot = (long)blockIdx.x + (long)b * H + kvh;
+  float* dst_o = ws + slot * (G * D);
+  float* dst_ml = ws + (long)nslots * (G * D) + slot * (G * 2);
   for (int i = tid; i < G * D; i += kDecThreads) {
     const int h = i / D, ch = i % D;
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) v = fmaf(ow[(w * G + h) * D + ch], wt[w * G + h], v);
-    dst_o[(long)h * splits * D + ch] = v;
+    dst_o[i] = v;
   }
   if (tid < G) {
     float l = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) l = fmaf(lw[w * G + tid], wt[w * G + tid], l);
-    dst_ml[(long)tid * splits * 2] = red[kDecWarps * G + tid];
-    dst_ml[(long)tid * splits * 2 + 1] = l;
+    dst_ml[2 * tid] = red[kDecWarps * G + tid];
+    dst_ml[2 * tid + 1] = l;
   }
-  pdl_trigger();
+  __syncthreads();  // the merge buffers alias the stages the next segment fills
+  };
+
+  // ---- walk the rows whose tiles meet [t0, t1), one chunk of rows at a time
+  long long base = 0;  // tiles per KV head of the rows before the chunk
+  for (int b0 = 0; b0 < cv.batch && base * H < t1; b0 += kDecThreads) {
+    long long x = x0, p = p0, tot = rows_total;
+    if (!one_chunk) {
+      const int r = b0 + tid;
+      x = r < cv.batch ? row_tiles(cv, r, max_ctx) : 0;
+      p = base + block_exclusive_scan<kDecThreads>(x, scan, &tot);
+    }
+    row_n[tid] = (int)x;
+    row_p[tid] = p;
+    __syncthreads();
+    // the prefixes never decrease: search the first row ending after t0
+    const int rows = min(kDecThreads, cv.batch - b0);
+    int lo = 0, hi = rows;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((row_p[mid] + row_n[mid]) * H > t0) hi = mid; else lo = mid + 1;
+    }
+    for (int i = lo; i < rows && row_p[i] * H < t1; ++i) {
+      const int n = row_n[i];
+      if (n == 0) continue;
+      b = b0 + i;
+      const long long rs = row_p[i] * H;  // first tile of the row
+      const int L = row_len(cv, b, max_ctx);
+      const int h_lo = t0 > rs ? (int)((t0 - rs) / n) : 0;
+      const int h_hi = (int)min((long long)(H - 1), (t1 - 1 - rs) / n);
+      for (kvh = h_lo; kvh <= h_hi; ++kvh) {
+        const long long us = rs + (long long)kvh * n;
+        t_begin = (int)(max(t0, us) - us) * kDecTile;
+        t_end = min((int)(min(t1, us + n) - us) * kDecTile, L);
+        row_slot = ((long)b * H + kvh) * cv.capacity;
+        segment();
+      }
+    }
+    base += tot;
+    __syncthreads();  // the row arrays are rewritten by the next chunk
+  }
 }
 
-// Launches decode_kernel for one compile-time shape (grid: splits x kv_heads x batch).
+// Sets the kernel's shared-memory attribute (once per device) and reports how
+// many of its CTAs fit on one SM.
 template <int D, int G, int KB, int VB, bool QJL>
-cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const void* q, int dtype,
-                                int q_heads, float scale_log2, const DecodePlan& plan,
-                                float* ws, cudaStream_t stream) {
+cudaError_t configure_shape(int* ctas_per_sm) {
   using Geo = DecodeGeom<D, G, KB, VB, QJL>;
   auto kern = decode_kernel<D, G, KB, VB, QJL>;
   static int configured_device = -1;
+  static int occupancy = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (configured_device != dev) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::total);
     if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occupancy, kern, kDecThreads, Geo::total);
+    if (e != cudaSuccess) return e;
     configured_device = dev;
   }
+  if (ctas_per_sm) *ctas_per_sm = occupancy;
+  return cudaSuccess;
+}
+
+// Launches decode_kernel for one compile-time shape (grid: plan.ctas CTAs).
+template <int D, int G, int KB, int VB, bool QJL>
+cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const void* q, int dtype,
+                                int q_heads, float scale_log2, int max_ctx,
+                                const DecodePlan& plan, float* ws, cudaStream_t stream) {
+  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
+  auto kern = decode_kernel<D, G, KB, VB, QJL>;
+  cudaError_t e = configure_shape<D, G, KB, VB, QJL>(nullptr);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.splits, cv.kv_heads, cv.batch);
+  cfg.gridDim = dim3(plan.ctas);
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = Geo::total;
   cfg.stream = stream;
@@ -719,26 +856,47 @@ cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const voi
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tb, cv, q, dtype, q_heads, scale_log2, plan.chunk,
-                            plan.splits, ws);
+  return cudaLaunchKernelEx(&cfg, kern, tb, cv, q, dtype, q_heads, scale_log2, max_ctx,
+                            plan.slots, ws);
 }
 
 // Per-head-dim dispatch over (group, k_bits, v_bits, qjl); instantiated in the
 // tq_decode_d<D>.cu translation units.
 template <int D>
+cudaError_t decode_occupancy_dim(const Tables& tb, int group, int* ctas_per_sm);
+
+template <int D>
+cudaError_t dispatch_occupancy_dim(const Tables& tb, int G, int* ctas_per_sm) {
+#define TQ_CASE(GG, KB, VB, QJ)                                             \
+  if (G == GG && tb.k_bits == KB && tb.v_bits == VB && (tb.qjl != 0) == QJ) \
+    return configure_shape<D, GG, KB, VB, QJ>(ctas_per_sm);
+#define TQ_BITS(GG, QJ) \
+  TQ_CASE(GG, 2, 2, QJ) TQ_CASE(GG, 2, 3, QJ) TQ_CASE(GG, 3, 3, QJ) TQ_CASE(GG, 3, 4, QJ) TQ_CASE(GG, 4, 4, QJ)
+#define TQ_GROUP(GG) TQ_BITS(GG, false) TQ_BITS(GG, true)
+  TQ_GROUP(1)
+  TQ_GROUP(2)
+  TQ_GROUP(4)
+  TQ_GROUP(8)
+#undef TQ_GROUP
+#undef TQ_BITS
+#undef TQ_CASE
+  return cudaErrorNotSupported;
+}
+
+template <int D>
 cudaError_t launch_decode_dim(const Tables& tb, const CacheView& cv, const void* q, int dtype,
-                              int q_heads, float scale_log2, const DecodePlan& plan, float* ws,
-                              cudaStream_t stream);
+                              int q_heads, float scale_log2, int max_ctx, const DecodePlan& plan,
+                              float* ws, cudaStream_t stream);
 
 template <int D>
 cudaError_t dispatch_decode_dim(const Tables& tb, const CacheView& cv, const void* q, int dtype,
-                                int q_heads, float scale_log2, const DecodePlan& plan, float* ws,
-                                cudaStream_t stream) {
+                                int q_heads, float scale_log2, int max_ctx,
+                                const DecodePlan& plan, float* ws, cudaStream_t stream) {
   const int G = q_heads / cv.kv_heads;
 #define TQ_CASE(GG, KB, VB, QJ)                                                               \
   if (G == GG && tb.k_bits == KB && tb.v_bits == VB && (tb.qjl != 0) == QJ)                   \
-    return launch_decode_shape<D, GG, KB, VB, QJ>(tb, cv, q, dtype, q_heads, scale_log2, plan, \
-                                                  ws, stream);
+    return launch_decode_shape<D, GG, KB, VB, QJ>(tb, cv, q, dtype, q_heads, scale_log2,     \
+                                                  max_ctx, plan, ws, stream);
 #define TQ_BITS(GG, QJ) \
   TQ_CASE(GG, 2, 2, QJ) TQ_CASE(GG, 2, 3, QJ) TQ_CASE(GG, 3, 3, QJ) TQ_CASE(GG, 3, 4, QJ) TQ_CASE(GG, 4, 4, QJ)
 #define TQ_GROUP(GG) TQ_BITS(GG, false) TQ_BITS(GG, true)

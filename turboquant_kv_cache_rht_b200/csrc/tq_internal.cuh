@@ -45,18 +45,32 @@ enum DType : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const void* k,
                                    const void* v, int dtype, int n_new, cudaStream_t stream);
 
-// Split of the context over CTAs for one decode call.
+// Work partition of one decode call.  Row b holds n_b = ceil(L_b / 64) token
+// tiles per KV head, L_b being seq_lens[b] clamped to [0, min(capacity,
+// max_ctx)].  The units u = b * kv_heads + h are laid end to end (unit (b, h)
+// covers tiles [kv_heads * P_b + h * n_b, ... + n_b), P_b = sum of n over the
+// rows before b), and CTA c of `ctas` takes tiles [c*T/ctas, (c+1)*T/ctas) of
+// the T in total.  The kernels compute this on the device from the lengths
+// they read there.  Each (CTA, unit) segment leaves one partial result in
+// workspace slot c + u; segments move monotonically in both c and u, so the
+// slots are distinct and `slots` = ctas + units - 1 bounds them.
 struct DecodePlan {
-  int splits;  // CTAs per (batch row, KV head)
-  int chunk;   // tokens per split (multiple of the token tile)
+  int ctas;
+  int slots;
 };
-DecodePlan plan_decode(int batch, int kv_heads, int max_ctx, int head_dim);
-size_t decode_workspace_bytes(const DecodePlan& plan, int batch, int q_heads, int head_dim);
+// At most `target_ctas` CTAs and no more than the tiles max_ctx allows.
+DecodePlan plan_decode(int batch, int kv_heads, int max_ctx, long target_ctas);
+// The most CTAs a launch uses (4 per SM of a 148-SM B200); the workspace for
+// it bounds the workspace of every launch.
+constexpr long kMaxTargetCtas = 148L * 4;
+size_t decode_workspace_bytes(const DecodePlan& plan, int q_heads, int kv_heads, int head_dim);
 
-// Returns cudaErrorNotSupported when no kernel is built for this shape.
+// Sizes the grid for one wave of the decode kernel at its real occupancy on
+// this device and launches decode + combine.  Returns cudaErrorNotSupported when no kernel is
+// built for this shape.
 cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, int dtype,
-                          int q_heads, float scale, const DecodePlan& plan, float* out,
-                          float* workspace, cudaStream_t stream);
+                          int q_heads, float scale, int max_ctx, float* out, float* workspace,
+                          cudaStream_t stream);
 bool decode_supported(int head_dim, int group, int k_bits, int v_bits, int qjl);
 
 // Stores `message` as this thread's last error and returns `status`.
