@@ -53,7 +53,12 @@ FALLBACK_HBM_GBS = 6650.0
 # sources change the figure no longer describes them and is reported as null.
 DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d128.cu", "tq_decode_d256.cu",
                   "tq_internal.cuh")
-DECODE_TRAFFIC: dict[str, tuple[int, str]] = {}
+DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
+    "gqa": (31746048, "c127026c84fdb290"),
+    "qjl": (566686976, "c127026c84fdb290"),
+    "long": (352887808, "c127026c84fdb290"),
+    "serving": (1102792192, "c127026c84fdb290"),
+}
 
 
 def decode_sources_digest() -> str:
@@ -312,26 +317,23 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         ctx_tokens += sum(lens)
     ms_max, bytes_all, tokens_all = reduce_over_ranks(ms, float(total_bytes), float(ctx_tokens), dev)
 
-    # ---- the decode call alone: events around each call, host queued ahead
-    dec_ms = []
-    app_ms = []
+    # ---- each call alone, back to back on the launching stream (host queued
+    #      ahead): one append per replica, then decode calls over the replicas
+    n_dec = max(st.replicas, 16)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     torch.cuda._sleep(2_000_000)
-    evs = []
+    ev[0].record(stream)
     for r in range(st.replicas):
-        a0, a1, d1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        c = st.caches[r]
-        a0.record(stream)
-        tq.tq_quantize_append(st.cb, c, st.k_new, st.v_new)
-        a1.record(stream)
-        tq.tq_decode_attention(st.cb, c, st.q, out=st.out, max_ctx=st.max_ctx, workspace=st.ws)
-        d1.record(stream)
-        evs.append((a0, a1, d1, [int(x) for x in st.lengths]))
+        tq.tq_quantize_append(st.cb, st.caches[r], st.k_new, st.v_new)
+    ev[1].record(stream)
+    ev[2].record(stream)
+    for i in range(n_dec):
+        tq.tq_decode_attention(st.cb, st.caches[i % st.replicas], st.q, out=st.out,
+                               max_ctx=st.max_ctx, workspace=st.ws)
+    ev[3].record(stream)
     torch.cuda.synchronize(dev)
-    for a0, a1, d1, _ in evs:
-        app_ms.append(a0.elapsed_time(a1))
-        dec_ms.append(a1.elapsed_time(d1))
-    dec_us = 1e3 * statistics.mean(dec_ms)
-    app_us = 1e3 * statistics.mean(app_ms)
+    app_us = 1e3 * ev[0].elapsed_time(ev[1]) / st.replicas
+    dec_us = 1e3 * ev[2].elapsed_time(ev[3]) / n_dec
     lens_now = [int(x) for x in st.caches[0].seq_lens.cpu()]
     dec_bytes = step_bytes(w, lens_now)["decode"]
 
