@@ -39,18 +39,24 @@ def _check_unit(cache, tb, b, h, k_all, v_all, qjl):
                               ek["rnorm16"].view(np.uint16)), "residual norms"
 
 
+# The encode kernel has two lane layouts, chosen by the append's total vector
+# count (keys and values of every row): up to 4096 vectors one vector per warp,
+# above that 32 channels per lane.  n = 37 and n = 700 (with B = 2, H = 3) fall
+# on either side, so every case runs through both.
 @pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("kb,vb", [(2, 2), (2, 3), (3, 3), (3, 4), (4, 4)])
 @pytest.mark.parametrize("qjl", [False, True])
-def test_codec_bit_exact(d, kb, vb, qjl):
-    B, H, n = 2, 3, 37
+@pytest.mark.parametrize("n", [37, 700])
+def test_codec_bit_exact(d, kb, vb, qjl, n):
+    B, H = 2, 3
+    assert (2 * B * H * n > 4096) == (n == 700)
     g = torch.Generator().manual_seed(d * 100 + kb * 10 + vb + qjl)
     k = torch.randn(B, H, n, d, generator=g)
     v = torch.randn(B, H, n, d, generator=g) * 3.0
     k[:, :, :, 5] *= 30.0                      # outlier channel
     cb = tq.Codebook(d, kb, vb, qjl, seed=42)
     tb = oracle_tables(d, kb, vb, qjl, 42)
-    cache = _run(cb, B, H, 64, [(k, v)])
+    cache = _run(cb, B, H, (n + 15) // 16 * 16, [(k, v)])
     assert cache.seq_lens.cpu().tolist() == [n] * B
     assert cache.append_sync.cpu().tolist() == [0] * B
     assert int(cache.status.item()) == 0
@@ -97,11 +103,15 @@ def test_adversarial_vectors():
             torch.linspace(-1000, 1000, d), torch.randn(d, generator=torch.Generator().manual_seed(1)) * 1e-20]
     k = torch.stack(rows)[None, None]                  # [1, 1, n, d]
     v = torch.flip(k, dims=[2]).contiguous()
-    for qjl in (False, True):
-        for kb, vb in ((2, 2), (3, 4), (4, 4)):
-            cb = tq.Codebook(d, kb, vb, qjl, seed=0)
-            cache = _run(cb, 1, H, 16, [(k, v)])
-            _check_unit(cache, oracle_tables(d, kb, vb, qjl, 0), 0, 0, k[0, 0], v[0, 0], qjl)
+    # the 7 rows alone (one vector per warp), and repeated 300 times (4200
+    # vectors: 32 channels per lane)
+    for reps in (1, 300):
+        kr, vr = k.repeat(1, 1, reps, 1), v.repeat(1, 1, reps, 1)
+        for qjl in (False, True):
+            for kb, vb in ((2, 2), (3, 4), (4, 4)):
+                cb = tq.Codebook(d, kb, vb, qjl, seed=0)
+                cache = _run(cb, 1, H, (7 * reps + 15) // 16 * 16, [(kr, vr)])
+                _check_unit(cache, oracle_tables(d, kb, vb, qjl, 0), 0, 0, kr[0, 0], vr[0, 0], qjl)
 
 
 def test_capacity_overflow_flags_and_skips():
