@@ -31,10 +31,12 @@
 //   signs : like keys, pairing bits (j, j+16) of a word so one shift places
 //           both sign bits of a half2 (+-1.0 needs no table)
 // Tiles of 64 tokens (one 16-token slab per warp) are staged by cp.async in a
-// 3-stage pipeline.  Each warp keeps its own online-softmax state; the four
-// warps are merged in a fixed order and each segment's partial (max, sum,
-// output) goes to the workspace, where the combine kernel merges the
-// partials of every unit and applies the inverse rotation.
+// 3-stage pipeline.  Each warp aggregates the values of its previous slab at
+// the top of its next one (from registers and the value table), so that work
+// overlaps the next slab's scoring.  Each warp keeps its own online-softmax
+// state; the four warps are merged in a fixed order and each segment's
+// partial (max, sum, output) goes to the workspace, where the combine kernel
+// merges the partials of every unit and applies the inverse rotation.
 #pragma once
 
 #include "tq_internal.cuh"
@@ -560,6 +562,32 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
   const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
 
+  // value aggregation of the warp's previous slab, run at the top of its next
+  // slab so that it overlaps that slab's score work (registers and the value
+  // table only: the stage it came from may already be refilled)
+  uint32_t pva[Geo::VCW], pvb[Geo::VCW], pvc[Geo::VCW], pvd[Geo::VCW], ppb[NT][2];
+#pragma unroll
+  for (int w = 0; w < Geo::VCW; ++w) pva[w] = pvb[w] = pvc[w] = pvd[w] = 0u;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) ppb[j][0] = ppb[j][1] = 0u;
+  auto aggregate = [&]() {
+    uint32_t y0[Geo::VCW], z0[Geo::VCW], y1[Geo::VCW], z1[Geo::VCW];
+    interleave_pairs<VB, Geo::VCW>(pva, pvb, y0, z0);
+    interleave_pairs<VB, Geo::VCW>(pvc, pvd, y1, z1);
+#pragma unroll
+    for (int mb = 0; mb < Geo::MBLK; ++mb) {
+      uint32_t e0, o0, e1, o1;
+      value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
+      value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma16816(acc[j][mb], a0, a1, a2, a3, ppb[j][0], ppb[j][1]);
+    }
+  };
+
   for (int it = 0; it < n_tiles; ++it) {
     cp_async_wait<1>();
     __syncthreads();
@@ -570,6 +598,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     const int n_valid = min(16, t_end - (t_begin + it * kDecTile + 16 * warp));
     if (n_valid <= 0) continue;
     const int r0 = 16 * warp;  // the warp's slab: rows r0 .. r0+15 of the stage
+    aggregate();               // O^T += V_hat^T . P^T of the previous slab, on the tensor cores
 
     // value code chunks of tokens 2q, 2q+1, 2q+8, 2q+9, loaded early so their
     // latency overlaps the score work
@@ -693,25 +722,21 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       pb[j][1] = __byte_perm(x1, x2, 0x7632);  // tokens 2q+8, 2q+9
     }
 
-    // ---- output: O^T += V_hat^T . P^T on the tensor cores
-    {
-      uint32_t y0[Geo::VCW], z0[Geo::VCW], y1[Geo::VCW], z1[Geo::VCW];
-      interleave_pairs<VB, Geo::VCW>(va, vb2, y0, z0);
-      interleave_pairs<VB, Geo::VCW>(vc, vd, y1, z1);
+    // ---- hand this slab's value codes and P to the next slab's aggregation
 #pragma unroll
-      for (int mb = 0; mb < Geo::MBLK; ++mb) {
-        uint32_t e0, o0, e1, o1;
-        value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
-        value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+    for (int w = 0; w < Geo::VCW; ++w) {
+      pva[w] = va[w];
+      pvb[w] = vb2[w];
+      pvc[w] = vc[w];
+      pvd[w] = vd[w];
+    }
 #pragma unroll
-        for (int j = 0; j < NT; ++j) mma16816(acc[j][mb], a0, a1, a2, a3, pb[j][0], pb[j][1]);
-      }
+    for (int j = 0; j < NT; ++j) {
+      ppb[j][0] = pb[j][0];
+      ppb[j][1] = pb[j][1];
     }
   }
+  aggregate();  // the warp's last slab
 
   // ---- epilogue: merge the four warps (fixed order) into the CTA's partial
 #pragma unroll
