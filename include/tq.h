@@ -140,6 +140,28 @@ tq_status tq_codebook_tables(const tq_codebook* cb, float* k_centroids, float* k
 tq_status tq_quantize_append(const tq_codebook* cb, const tq_cache* cache, const void* k,
                              const void* v, tq_dtype dtype, int n_new, void* stream);
 
+/* Converts an existing dense K/V cache into the compressed one: the prefill of
+ * a whole context at once, or the conversion of a cache filled by an
+ * unquantized model ("How to Use TurboQuant with the MLX-VLM Python API",
+ * "What is TurboQuant?": a filled KVCache is converted by from_cache).  Every
+ * vector goes through the same codec as tq_quantize_append.
+ * k, v : DEVICE, dtype `dtype`; element (b, h, t, i) of k is
+ *        k[b*stride_b + h*stride_h + t*stride_t + i] (strides in elements,
+ *        the channel stride is 1; v uses the same strides), so both
+ *        [batch][kv_heads][T][d] and [batch][T][kv_heads][d] caches are read in
+ *        place.  Every stride times the element size must be a multiple of 16
+ *        bytes, and k and v 16-byte aligned.
+ * lengths : DEVICE int32 [batch], tokens of row b to convert (t < lengths[b]).
+ * max_len : host upper bound of every lengths[b] (it sizes the grid).
+ * Row b's slots [0, lengths[b]) are overwritten and seq_lens[b] is set to
+ * lengths[b] (earlier contents of the row are discarded).  A row longer than
+ * `capacity` is skipped and sets TQ_FLAG_CAPACITY; a length above max_len
+ * converts the first max_len tokens and sets TQ_FLAG_MAXCTX; a negative
+ * length counts as 0.  No counterpart of append_sync is used. */
+tq_status tq_quantize_cache(const tq_codebook* cb, const tq_cache* cache, const void* k,
+                            const void* v, tq_dtype dtype, int64_t stride_b, int64_t stride_h,
+                            int64_t stride_t, const int32_t* lengths, int max_len, void* stream);
+
 /* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes):
  * (min(592, U * ceil(max_ctx / 64)) + U - 1) * (q_heads / kv_heads) *
  * (head_dim + 2) * 4, U = batch * kv_heads -- one partial result per (CTA,

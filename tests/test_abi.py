@@ -97,6 +97,28 @@ def test_append_validation():
                                      None) == tq.TQ_ERR_INVALID
 
 
+def _convert(cb, cache, k=1 << 12, v=1 << 13, dtype=1, strides=(2 * 64 * 128, 64 * 128, 128),
+             lengths=1 << 14, max_len=64):
+    return tq.lib.tq_quantize_cache(cb.handle, C.byref(cache), k, v, dtype, *strides, lengths,
+                                    max_len, None)
+
+
+def test_convert_validation():
+    """Rejected before any launch (the pointers are fake; no GPU is touched)."""
+    cb = tq.Codebook(128, 3, 4)
+    assert _convert(cb, _fake_cache(capacity=40)) == tq.TQ_ERR_INVALID        # capacity % 16
+    assert _convert(cb, _fake_cache(), dtype=7) == tq.TQ_ERR_INVALID
+    assert _convert(cb, _fake_cache(), max_len=-1) == tq.TQ_ERR_INVALID
+    assert _convert(cb, _fake_cache(), max_len=0) == tq.TQ_OK                 # no-op, no launch
+    assert _convert(cb, _fake_cache(), k=0) == tq.TQ_ERR_INVALID
+    assert _convert(cb, _fake_cache(), lengths=0) == tq.TQ_ERR_INVALID
+    assert _convert(cb, _fake_cache(), lengths=(1 << 14) + 2) == tq.TQ_ERR_INVALID   # misaligned
+    assert _convert(cb, _fake_cache(), k=(1 << 12) + 8) == tq.TQ_ERR_INVALID         # misaligned
+    assert _convert(cb, _fake_cache(), strides=(1, 128, 128)) == tq.TQ_ERR_INVALID   # 2 bytes
+    assert _convert(cb, _fake_cache(), strides=(64, 128, 4)) == tq.TQ_ERR_INVALID    # 8 bytes
+    assert _convert(cb, _fake_cache(), strides=(-128, 128, 128)) == tq.TQ_ERR_INVALID
+
+
 def _decode(cb, cache, q_heads=4, max_ctx=64, ws=1 << 14, ws_bytes=1 << 30, scale=0.0, q=1 << 12):
     return tq.lib.tq_decode_attention(cb.handle, C.byref(cache), q, 1, q_heads, scale, max_ctx,
                                       1 << 13, ws, ws_bytes, None)

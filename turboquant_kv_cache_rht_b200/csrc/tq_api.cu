@@ -255,6 +255,30 @@ tq_status tq_quantize_append(const tq_codebook* cb, const tq_cache* cache, const
                      "quantize-append launch");
 }
 
+tq_status tq_quantize_cache(const tq_codebook* cb, const tq_cache* cache, const void* k,
+                            const void* v, tq_dtype dtype, int64_t stride_b, int64_t stride_h,
+                            int64_t stride_t, const int32_t* lengths, int max_len, void* stream) {
+  tq_status st = check_cache(cb, cache);
+  if (st != TQ_OK) return st;
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (max_len < 0) return fail(TQ_ERR_INVALID, "max_len %d is negative", max_len);
+  if (max_len == 0) return ok();
+  if (!k || !v || !lengths) return fail(TQ_ERR_INVALID, "k, v or lengths is NULL");
+  if (stride_b < 0 || stride_h < 0 || stride_t < 0)
+    return fail(TQ_ERR_INVALID, "negative stride");
+  const int64_t esz = dtype == TQ_F32 ? 4 : 2;
+  if ((stride_b * esz) % 16 || (stride_h * esz) % 16 || (stride_t * esz) % 16)
+    return fail(TQ_ERR_INVALID, "strides (%lld, %lld, %lld) are not multiples of 16 bytes",
+                (long long)stride_b, (long long)stride_h, (long long)stride_t);
+  if (!aligned16(k) || !aligned16(v)) return fail(TQ_ERR_INVALID, "k and v must be 16-byte aligned");
+  if ((uintptr_t)lengths % 4) return fail(TQ_ERR_INVALID, "lengths must be 4-byte aligned");
+  return cuda_status(tq::launch_quantize_cache(cb->tables, view_of(cache), k, v, (int)dtype,
+                                               stride_b, stride_h, stride_t, lengths, max_len,
+                                               (cudaStream_t)stream),
+                     "quantize-cache launch");
+}
+
 size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
                                  int max_ctx) {
   if (!cb || batch <= 0 || q_heads <= 0 || kv_heads <= 0 || max_ctx < 0 ||

@@ -44,6 +44,11 @@ enum DType : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
 cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const void* k,
                                    const void* v, int dtype, int n_new, cudaStream_t stream);
+// Dense cache (strides in elements) -> compressed cache, lengths[b] tokens per row.
+cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const void* k,
+                                  const void* v, int dtype, long stride_b, long stride_h,
+                                  long stride_t, const int32_t* lengths, int max_len,
+                                  cudaStream_t stream);
 
 // Work partition of one decode call.  Row b holds n_b = ceil(L_b / 64) token
 // tiles per KV head, L_b being seq_lens[b] clamped to [0, min(capacity,

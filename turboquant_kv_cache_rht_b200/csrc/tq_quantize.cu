@@ -313,6 +313,68 @@ __global__ void __launch_bounds__(kAppendThreads)
   pdl_trigger();
 }
 
+// Conversion of a dense cache.  Grid: (2 * blocks_per_kind, batch) as for the
+// append; the vectors (h, t) of a row are numbered with t outermost when the
+// input's head stride is the smaller one (a [batch][T][heads][d] cache) and
+// with h outermost otherwise, so consecutive lanes read consecutive memory.
+template <int D, typename T, int E>
+__global__ void __launch_bounds__(kAppendThreads)
+    quantize_convert_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
+                            const T* __restrict__ kin, const T* __restrict__ vin, long stride_b,
+                            long stride_h, long stride_t, const int32_t* __restrict__ lengths,
+                            int max_len, int blocks_per_kind, int heads_inner) {
+  constexpr int GL = D / E;
+  constexpr int VPB = kAppendThreads / GL;
+  __shared__ float s_kcent[16];
+  __shared__ uint32_t s_pack[kAppendWarps][E < 32 ? D / 8 + 1 : 1];
+
+  const int tid = threadIdx.x, lane = tid & 31, g = lane & (GL - 1);
+  if (tid < 16) s_kcent[tid] = tb.k_cent[tid];
+  const int b = blockIdx.y, H = cv.kv_heads;
+  const bool is_v = (int)blockIdx.x >= blocks_per_kind;
+  const long r = (long)(blockIdx.x - (is_v ? blocks_per_kind : 0)) * VPB + tid / GL;
+  const bool in_grid = r < (long)H * max_len;
+  const int h = !in_grid ? 0 : heads_inner ? (int)(r % H) : (int)(r / max_len);
+  const int t = !in_grid ? 0 : heads_inner ? (int)(r / H) : (int)(r % max_len);
+
+  pdl_wait();
+  const int asked = max(lengths[b], 0);
+  const int len = min(asked, max_len);
+  const bool fits = len <= cv.capacity;
+  if (tid == 0 && blockIdx.x == 0) {
+    if (asked > max_len) atomicOr(cv.status, (int)kFlagMaxCtx);
+    if (fits) cv.seq_lens[b] = len;  // no block of this grid reads seq_lens
+    else atomicOr(cv.status, (int)kFlagCapacity);
+  }
+  const bool valid = fits && in_grid && t < len;
+  __syncthreads();  // s_kcent
+
+  if (__any_sync(kFull, valid)) {
+    float u[E];
+    const T* src = (is_v ? vin : kin) + b * stride_b + h * stride_h + t * stride_t + g * E;
+    if (valid) {
+      load_elems<E>(src, u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) u[e] = 0.f;
+    }
+    const long slot = ((long)b * H + h) * cv.capacity + t;
+    const int bits = is_v ? tb.v_bits : tb.k_bits;
+    uint8_t* codes = (is_v ? cv.v_codes : cv.k_codes) + slot * (long)(bits * D / 8);
+    uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot;
+    uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
+    uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
+    uint32_t* pack = s_pack[tid >> 5];
+    if (bits == 2)
+      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    else if (bits == 3)
+      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    else
+      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+  }
+  pdl_trigger();
+}
+
 // Appends of at most this many vectors in all (keys and values of every row)
 // take the one-vector-per-warp layout: they are too few to fill the GPU, so
 // latency rules; larger ones take the 32-channels-per-lane layout.
@@ -347,6 +409,51 @@ cudaError_t launch_typed(const Tables& tb, const CacheView& cv, const void* k, c
   return launch_layout<D, T, 32>(tb, cv, k, v, n_new, stream);
 }
 
+template <int D, typename T, int E>
+cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const void* k,
+                                  const void* v, long sb, long sh, long st,
+                                  const int32_t* lengths, int max_len, cudaStream_t stream) {
+  constexpr int VPB = kAppendThreads / (D / E);
+  const long per_kind = (long)cv.kv_heads * max_len;
+  const long blocks_per_kind = std::max<long>(1, (per_kind + VPB - 1) / VPB);
+  if (2 * blocks_per_kind > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * blocks_per_kind), (unsigned)cv.batch);
+  cfg.blockDim = dim3(kAppendThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_convert_kernel<D, T, E>, tb, cv,
+                            static_cast<const T*>(k), static_cast<const T*>(v), sb, sh, st,
+                            lengths, max_len, (int)blocks_per_kind, sh < st ? 1 : 0);
+}
+
+template <int D, typename T>
+cudaError_t launch_convert_typed(const Tables& tb, const CacheView& cv, const void* k,
+                                 const void* v, long sb, long sh, long st, const int32_t* lengths,
+                                 int max_len, cudaStream_t stream) {
+  const long vectors = 2L * cv.batch * cv.kv_heads * max_len;
+  if (vectors <= kLatencyVectors)
+    return launch_convert_layout<D, T, D / 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+  return launch_convert_layout<D, T, 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+}
+
+template <int D>
+cudaError_t launch_convert_dim(const Tables& tb, const CacheView& cv, const void* k, const void* v,
+                               int dtype, long sb, long sh, long st, const int32_t* lengths,
+                               int max_len, cudaStream_t stream) {
+  switch (dtype) {
+    case kF32: return launch_convert_typed<D, float>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+    case kBF16:
+      return launch_convert_typed<D, __nv_bfloat16>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+    case kF16: return launch_convert_typed<D, __half>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int D>
 cudaError_t launch_dim(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                        int dtype, int n_new, cudaStream_t stream) {
@@ -365,6 +472,21 @@ cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const 
   switch (tb.d) {
     case 128: return launch_dim<128>(tb, cv, k, v, dtype, n_new, stream);
     case 256: return launch_dim<256>(tb, cv, k, v, dtype, n_new, stream);
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const void* k,
+                                  const void* v, int dtype, long stride_b, long stride_h,
+                                  long stride_t, const int32_t* lengths, int max_len,
+                                  cudaStream_t stream) {
+  switch (tb.d) {
+    case 128:
+      return launch_convert_dim<128>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                     max_len, stream);
+    case 256:
+      return launch_convert_dim<256>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                     max_len, stream);
   }
   return cudaErrorNotSupported;
 }

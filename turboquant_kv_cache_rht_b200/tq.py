@@ -27,7 +27,7 @@ TQ_OK, TQ_ERR_INVALID, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_CAPACITY, TQ_ERR_
 TQ_FLAG_CAPACITY = 1
 TQ_FLAG_MAXCTX = 2
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
-EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append",
+EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append", "tq_quantize_cache",
            "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_noalloc",
            "tq_free", "tq_last_error")
 
@@ -56,6 +56,9 @@ lib.tq_codebook_tables.restype = C.c_int
 lib.tq_quantize_append.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_void_p,
                                    C.c_int, C.c_int, C.c_void_p]
 lib.tq_quantize_append.restype = C.c_int
+lib.tq_quantize_cache.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_void_p, C.c_int,
+                                  C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_int, C.c_void_p]
+lib.tq_quantize_cache.restype = C.c_int
 lib.tq_decode_workspace_bytes.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int]
 lib.tq_decode_workspace_bytes.restype = C.c_size_t
 lib.tq_decode_attention.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_int, C.c_int,
@@ -185,6 +188,30 @@ def tq_quantize_append(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Ten
     _check(lib.tq_quantize_append(cb.handle, C.byref(cs), k.data_ptr(), v.data_ptr(),
                                   _dtype_code(k), k.shape[2], _stream_ptr(stream)),
            "tq_quantize_append")
+
+
+def tq_quantize_cache(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Tensor,
+                      lengths: torch.Tensor | None = None, stream=None) -> None:
+    """Convert a dense cache: k, v are [batch, kv_heads, T, head_dim] CUDA tensors
+    of one dtype with unit channel stride and any other strides (a view of a
+    [batch, T, kv_heads, head_dim] cache transposed works in place); lengths is
+    an int32 CUDA tensor [batch] (default: T for every row).  Sets seq_lens."""
+    if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
+        raise ValueError("k and v must be [batch, kv_heads, T, head_dim] of one dtype")
+    if k.stride() != v.stride() or k.stride(3) != 1:
+        raise ValueError("k and v must share strides, with unit channel stride")
+    if k.shape[0] != cache.batch or k.shape[1] != cache.kv_heads or k.shape[3] != cb.head_dim:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match the cache")
+    T = k.shape[2]
+    if lengths is None:
+        lengths = torch.full((cache.batch,), T, dtype=torch.int32, device=k.device)
+    if lengths.dtype != torch.int32 or lengths.shape != (cache.batch,) or not lengths.is_contiguous():
+        raise ValueError("lengths must be a contiguous int32 tensor [batch]")
+    cs = cache.struct()
+    _check(lib.tq_quantize_cache(cb.handle, C.byref(cs), k.data_ptr(), v.data_ptr(), _dtype_code(k),
+                                 k.stride(0), k.stride(1), k.stride(2), lengths.data_ptr(), T,
+                                 _stream_ptr(stream)),
+           "tq_quantize_cache")
 
 
 def tq_decode_workspace_bytes(cb: Codebook, batch: int, q_heads: int, kv_heads: int,
