@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
 the CPU-baseline legs of ``bench.py``, never by the product path.  It shares no
-code, table or constant generator with the CUDA library; it imports numpy and the
-Python standard library only.
+code, table or constant generator with the CUDA library; it imports numpy, the
+Python standard library and, for the unit-sphere codebook only, scipy.special.
 
 Sources, cited by page title and section:
 
@@ -206,6 +206,84 @@ def codebook(bits: int) -> tuple[np.ndarray, np.ndarray]:
     """
     levels = 1 << bits
     c64, _ = lloyd_max_gaussian(levels)
+    half = levels // 2
+    pos = np.array([(c64[half + j] - c64[half - 1 - j]) / 2 for j in range(half)],
+                   dtype=np.float32)
+    cent = np.concatenate([-pos[::-1], pos]).astype(np.float32)
+    bnd = ((cent[:-1] + cent[1:]) * np.float32(0.5)).astype(np.float32)
+    return cent, bnd
+
+
+# ---------------------------------------------------------------------------
+# Codebook for the exact distribution of a rotated coordinate.  [P3]'s
+# introduction calls the rotated coordinates near-Gaussian, which is what the
+# N(0,1) codebook above assumes.  Exactly: for a fixed vector x, each
+# coordinate of R x / ||x|| is a coordinate of a uniformly random unit vector
+# of R^d, so z = sqrt(d) * (R x)_i / ||x|| has density
+#     f_d(z) = C_d * (1 - z^2/d)^((d-3)/2)  on |z| < sqrt(d),
+#     C_d = Gamma(d/2) / (sqrt(pi d) Gamma((d-1)/2)),
+# and z^2/d ~ Beta(1/2, (d-1)/2).  f_d tends to the N(0,1) density as d grows.
+
+def sphere_density(z: float, d: int) -> float:
+    if abs(z) >= math.sqrt(d):
+        return 0.0
+    c = math.exp(math.lgamma(d / 2) - math.lgamma((d - 1) / 2)) / math.sqrt(math.pi * d)
+    return c * (1.0 - z * z / d) ** ((d - 3) / 2)
+
+
+def _sphere_upper_tail(z: float, d: int) -> float:
+    """P(Z > z) for z >= 0: half of P(Z^2/d > z^2/d) (the complemented
+    regularized incomplete beta function, so no tail cancels)."""
+    from scipy.special import betaincc
+    if z >= math.sqrt(d):
+        return 0.0
+    return 0.5 * float(betaincc(0.5, (d - 1) / 2, z * z / d))
+
+
+def sphere_mass(a: float, b: float, d: int) -> float:
+    """P(a < Z < b) for the scaled coordinate Z of a random unit vector of R^d."""
+    if a >= 0.0:
+        return _sphere_upper_tail(a, d) - _sphere_upper_tail(b, d)
+    if b <= 0.0:
+        return _sphere_upper_tail(-b, d) - _sphere_upper_tail(-a, d)
+    return 1.0 - _sphere_upper_tail(-a, d) - _sphere_upper_tail(b, d)
+
+
+def sphere_first_moment(a: float, b: float, d: int) -> float:
+    """Integral of z f_d(z) over (a, b): an antiderivative of z (1 - z^2/d)^k is
+    -(d / (2 (k + 1))) (1 - z^2/d)^(k + 1), here with k = (d - 3)/2."""
+    r = math.sqrt(d)
+    a, b = max(a, -r), min(b, r)
+    c = math.exp(math.lgamma(d / 2) - math.lgamma((d - 1) / 2)) / math.sqrt(math.pi * d)
+    g = lambda z: max(0.0, 1.0 - z * z / d) ** ((d - 1) / 2)
+    return c * d / (d - 1) * (g(a) - g(b))
+
+
+def sphere_cell_mean(a: float, b: float, d: int) -> float:
+    """E[Z | a < Z < b]."""
+    return sphere_first_moment(a, b, d) / sphere_mass(a, b, d)
+
+
+def lloyd_max_sphere(levels: int, d: int, init=None, tol: float = 1e-14,
+                     max_iter: int = 1_000_000) -> tuple[np.ndarray, int]:
+    """Lloyd's iteration (midpoint boundaries, conditional-mean centroids) for
+    the density f_d; starts from the N(0,1) solution unless ``init`` is given."""
+    c = [float(t) for t in (lloyd_max_gaussian(levels)[0] if init is None else init)]
+    for it in range(1, max_iter + 1):
+        edges = [-math.inf] + [(c[j] + c[j + 1]) / 2 for j in range(levels - 1)] + [math.inf]
+        new = [sphere_cell_mean(edges[j], edges[j + 1], d) for j in range(levels)]
+        moved = max(abs(n - o) for n, o in zip(new, c))
+        c = new
+        if moved < tol:
+            return np.array(c, np.float64), it
+    raise RuntimeError("Lloyd-Max iteration did not converge")
+
+
+def sphere_codebook(bits: int, d: int) -> tuple[np.ndarray, np.ndarray]:
+    """(centroids, boundaries) in float32 for the density f_d, made odd-symmetric
+    and rounded exactly as ``codebook`` does for N(0,1)."""
+    levels = 1 << bits
+    c64, _ = lloyd_max_sphere(levels, d)
     half = levels // 2
     pos = np.array([(c64[half + j] - c64[half - 1 - j]) / 2 for j in range(half)],
                    dtype=np.float32)
