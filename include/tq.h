@@ -59,18 +59,33 @@ typedef enum {
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 
+/* Codebook choices (tq_params.codebook).
+ *   TQ_CODEBOOK_GAUSSIAN : Lloyd-Max quantizer of N(0, 1), the pages' reading
+ *       of the rotated coordinates as near-Gaussian ("How to Use TurboQuant
+ *       ...", "What is TurboQuant?": _codebook; "mlx-turboquant" README).
+ *   TQ_CODEBOOK_SPHERE : Lloyd-Max quantizer of their exact distribution: for a
+ *       fixed x, sqrt(d) (R x)_i / ||x|| is sqrt(d) times a coordinate of a
+ *       uniformly random unit vector of R^d, with density proportional to
+ *       (1 - z^2/d)^((d-3)/2) on |z| < sqrt(d); it depends on head_dim and
+ *       tends to N(0, 1) as head_dim grows. */
+#define TQ_CODEBOOK_GAUSSIAN 0
+#define TQ_CODEBOOK_SPHERE 1
+
 /* Codec parameters.
  *   head_dim : d, 128 or 256 (64 is reported as TQ_ERR_UNSUPPORTED)
  *   k_bits, v_bits : code widths in {2, 3, 4} ("3.5 bits" = 3 and 4)
  *   qjl      : 1 = keys also carry the 1-bit QJL residual sketch
  *   seed     : seeds the sign vectors of R (and of R2 = RHT2 for QJL).  One R
- *              is shared by keys, values, all heads and all batch rows. */
+ *              is shared by keys, values, all heads and all batch rows.
+ *   codebook : TQ_CODEBOOK_GAUSSIAN (0, the default when zero-initialized) or
+ *              TQ_CODEBOOK_SPHERE. */
 typedef struct {
   int head_dim;
   int k_bits;
   int v_bits;
   int qjl;
   uint64_t seed;
+  int codebook;
 } tq_params;
 
 /* Bytes stored per cached vector, in each per-vector array of tq_cache. */
@@ -108,10 +123,11 @@ typedef struct {
 } tq_cache;
 
 /* Builds the codebooks and rotation signs for `params` (host work only: no
- * GPU is needed).  Codebook: the Lloyd-Max MSE quantizer of N(0, 1) with
- * 2^bits levels, solved in double precision, made exactly odd-symmetric and
- * rounded to float32; boundaries are the float32 midpoints of adjacent
- * centroids ("How to Use TurboQuant ...", "What is TurboQuant?": _codebook).
+ * GPU is needed).  Codebook: the Lloyd-Max MSE quantizer with 2^bits levels of
+ * N(0, 1) or of the exact rotated-coordinate distribution (params->codebook),
+ * solved in double precision, made exactly odd-symmetric and rounded to
+ * float32; boundaries are the float32 midpoints of adjacent centroids ("How
+ * to Use TurboQuant ...", "What is TurboQuant?": _codebook).
  * Signs: channel i of D1 is -1 when the top bit of the i-th SplitMix64 output
  * from state `seed` is set; D2 uses state seed ^ 0x9E3779B97F4A7C15.
  * On success *out owns the tables (release with tq_free) and *layout, if not

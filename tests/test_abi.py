@@ -40,6 +40,21 @@ def test_tables_equal_oracle_bit_for_bit(d, kb, vb, seed):
     assert np.array_equal(t["signs2"].numpy(), o.rotation_signs(seed, d, second=True))
 
 
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb,vb", [(2, 2), (3, 4), (4, 4), (2, 3), (3, 3)])
+def test_sphere_tables_equal_oracle_bit_for_bit(d, kb, vb):
+    """The host solves the sphere codebook with its own integration (Gauss-Legendre
+    cell masses), the oracle with the incomplete beta function; the float32 tables
+    must agree bit for bit."""
+    cb = tq.Codebook(d, kb, vb, codebook="sphere")
+    t = cb.tables()
+    for bits, c_name, b_name in ((kb, "k_centroids", "k_boundaries"), (vb, "v_centroids", "v_boundaries")):
+        cent, bnd = o.sphere_codebook(bits, d)
+        assert np.array_equal(t[c_name].numpy().view(np.uint32), cent.view(np.uint32))
+        assert np.array_equal(t[b_name].numpy().view(np.uint32), bnd.view(np.uint32))
+    assert not np.array_equal(t["k_centroids"].numpy(), o.codebook(kb)[0])   # differs from N(0,1)
+
+
 def test_layout_bytes():
     cb = tq.Codebook(128, 3, 4, qjl=True)
     assert (cb.layout.k_code_bytes, cb.layout.v_code_bytes, cb.layout.k_sign_bytes) == (48, 64, 16)
@@ -48,11 +63,11 @@ def test_layout_bytes():
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(head_dim=512), dict(k_bits=1),
-                                 dict(v_bits=5), dict(qjl=2)])
+                                 dict(v_bits=5), dict(qjl=2), dict(codebook=2), dict(codebook=-1)])
 def test_codebook_rejects_bad_params(bad):
-    p = dict(head_dim=128, k_bits=3, v_bits=4, qjl=0, seed=0)
+    p = dict(head_dim=128, k_bits=3, v_bits=4, qjl=0, seed=0, codebook=0)
     p.update(bad)
-    params = tq.tq_params(p["head_dim"], p["k_bits"], p["v_bits"], p["qjl"], p["seed"])
+    params = tq.tq_params(p["head_dim"], p["k_bits"], p["v_bits"], p["qjl"], p["seed"], p["codebook"])
     h = C.c_void_p()
     assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_ERR_INVALID
     assert not h.value

@@ -65,6 +65,23 @@ def test_codec_bit_exact(d, kb, vb, qjl, n):
             _check_unit(cache, tb, b, h, k[b, h], v[b, h], qjl)
 
 
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb,vb,qjl", [(2, 2, True), (3, 4, False), (4, 4, True)])
+@pytest.mark.parametrize("n", [37, 700])
+def test_codec_bit_exact_sphere_codebook(d, kb, vb, qjl, n):
+    """The codec with the head_dim-specific sphere codebook (both lane layouts)."""
+    B, H = 2, 3
+    g = torch.Generator().manual_seed(7 * d + kb + n)
+    k = torch.randn(B, H, n, d, generator=g).bfloat16()
+    v = torch.randn(B, H, n, d, generator=g).bfloat16()
+    cb = tq.Codebook(d, kb, vb, qjl, seed=5, codebook="sphere")
+    tb = oracle_tables(d, kb, vb, qjl, 5, codebook="sphere")
+    cache = _run(cb, B, H, (n + 15) // 16 * 16, [(k, v)])
+    for b in range(B):
+        for h in range(H):
+            _check_unit(cache, tb, b, h, k[b, h], v[b, h], qjl)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 def test_input_dtypes(dtype):
     d, B, H, n = 128, 1, 2, 16

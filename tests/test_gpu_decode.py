@@ -133,6 +133,27 @@ def test_deterministic_and_partition_independent():
     assert_rows_close(c[2, 5 * G:6 * G].cpu().numpy(), ref)
 
 
+def test_sphere_codebook_decode():
+    d, G, B, Hkv = 128, 4, 2, 2
+    lengths = [300, 129]
+    g = torch.Generator().manual_seed(31)
+    k = torch.randn(B, Hkv, 300, d, generator=g).bfloat16()
+    v = torch.randn(B, Hkv, 300, d, generator=g).bfloat16()
+    q = torch.randn(B, Hkv * G, d, generator=g).bfloat16()
+    cb = tq.Codebook(d, 3, 4, True, seed=6, codebook="sphere")
+    cache = tq.Cache(cb, B, Hkv, 304, "cuda")
+    tq.tq_quantize_append(cb, cache, k.cuda(), v.cuda())
+    cache.seq_lens.copy_(torch.tensor(lengths, dtype=torch.int32))
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=304).cpu()
+    tb = oracle_tables(d, 3, 4, True, 6, codebook="sphere")
+    for b in range(B):
+        for h in range(Hkv):
+            n = lengths[b]
+            ek, ev = oracle_encode_unit(tb, k[b, h, :n], v[b, h, :n])
+            ref = oracle_decode_unit(tb, q[b, h * G:(h + 1) * G], ek, ev)
+            assert_rows_close(out[b, h * G:(h + 1) * G].numpy(), ref, what=f"({b},{h})")
+
+
 def test_many_ragged_rows():
     # 300 rows (more than one 128-row chunk of the decode's schedule and one
     # 256-row pass of the combine's), a quarter of them empty, lengths 0..200:

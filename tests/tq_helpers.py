@@ -11,9 +11,10 @@ import oracle as o
 DEC_TOL = 2e-3   # decode: per row, max |gpu - oracle| <= DEC_TOL * max |oracle|
 
 
-def oracle_tables(head_dim, k_bits, v_bits, qjl, seed):
-    ck, bk = o.codebook(k_bits)
-    cv, bv = o.codebook(v_bits)
+def oracle_tables(head_dim, k_bits, v_bits, qjl, seed, codebook="gaussian"):
+    book = (lambda b: o.codebook(b)) if codebook == "gaussian" else (lambda b: o.sphere_codebook(b, head_dim))
+    ck, bk = book(k_bits)
+    cv, bv = book(v_bits)
     s1 = o.rotation_signs(seed, head_dim)
     s2 = o.rotation_signs(seed, head_dim, second=True) if qjl else None
     return dict(ck=ck, bk=bk, cv=cv, bv=bv, s1=s1, s2=s2, k_bits=k_bits, v_bits=v_bits)

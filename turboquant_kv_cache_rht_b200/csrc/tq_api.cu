@@ -3,6 +3,7 @@
 #include "../../include/tq.h"
 #include "tq_internal.cuh"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -57,33 +58,122 @@ double normal_mass(double lo, double hi) {
   return 1.0 - normal_tail(-lo) - normal_tail(hi);
 }
 
-bool lloyd_max(int levels, double* level_out) {
-  double lv[16], next[16], edge[17];
-  for (int j = 0; j < levels; ++j) lv[j] = -2.0 + 4.0 * (j + 0.5) / levels;
+double normal_cell_mean(double lo, double hi) {
+  return (normal_density(lo) - normal_density(hi)) / normal_mass(lo, hi);
+}
+
+// The exact distribution of a rotated coordinate.  For a fixed x, each
+// coordinate of R x / ||x|| is a coordinate of a uniformly random unit vector
+// of R^d, so Z = sqrt(d) (R x)_i / ||x|| has density
+// f(z) = C_d (1 - z^2/d)^((d-3)/2) on |z| < sqrt(d), C_d = Gamma(d/2) /
+// (sqrt(pi d) Gamma((d-1)/2)); the rotated coordinates are only near-Gaussian
+// ("mlx-turboquant" README, introduction).  Cell masses are integrated
+// directly (composite 10-point Gauss-Legendre on pieces at most 1/4 wide,
+// compensated sums), so a small outer cell is not the difference of two
+// nearly equal cumulative integrals.
+struct Sphere {
+  int d;
+  double c;  // C_d
+};
+
+struct GaussLegendre10 {
+  double x[10], w[10];
+  GaussLegendre10() {  // roots of the Legendre polynomial P_10 by Newton's method
+    for (int i = 0; i < 10; ++i) {
+      double z = std::cos(M_PI * (i + 0.75) / 10.5), dp = 1.0;
+      for (int it = 0; it < 100; ++it) {
+        double p0 = 1.0, p1 = z;  // P_0, P_1, then the three-term recurrence
+        for (int k = 2; k <= 10; ++k) {
+          const double pk = ((2 * k - 1) * z * p1 - (k - 1) * p0) / k;
+          p0 = p1;
+          p1 = pk;
+        }
+        dp = 10 * (z * p1 - p0) / (z * z - 1.0);
+        const double step = p1 / dp;
+        z -= step;
+        if (std::fabs(step) < 1e-16) break;
+      }
+      x[i] = z;
+      w[i] = 2.0 / ((1.0 - z * z) * dp * dp);
+    }
+  }
+};
+
+// (1 - z^2/d)^k as exp(k log1p(-z^2/d)): a power of the rounded base would
+// carry k times the base's rounding error, which is what limits Lloyd's
+// iteration near its tolerance.
+double sphere_power(double z, int d, double k) {
+  const double x = z * z / d;
+  return x >= 1.0 ? 0.0 : std::exp(k * std::log1p(-x));
+}
+
+double sphere_density(const Sphere& sp, double z) { return sp.c * sphere_power(z, sp.d, (sp.d - 3) / 2.0); }
+
+double sphere_mass(const Sphere& sp, double lo, double hi) {
+  static const GaussLegendre10 gl;
+  const double r = std::sqrt((double)sp.d);
+  lo = std::fmax(lo, -r);
+  hi = std::fmin(hi, r);
+  if (!(hi > lo)) return 0.0;
+  const int pieces = std::max(1, (int)std::ceil((hi - lo) * 4.0));
+  const double h = (hi - lo) / pieces;
+  double sum = 0.0, comp = 0.0;  // Kahan summation
+  for (int p = 0; p < pieces; ++p) {
+    const double mid = lo + (p + 0.5) * h;
+    for (int i = 0; i < 10; ++i) {
+      const double term = gl.w[i] * sphere_density(sp, mid + 0.5 * h * gl.x[i]) * 0.5 * h - comp;
+      const double next = sum + term;
+      comp = (next - sum) - term;
+      sum = next;
+    }
+  }
+  return sum;
+}
+
+// Integral of z f(z) over (lo, hi): an antiderivative of z (1 - z^2/d)^k is
+// -(d / (2 (k + 1))) (1 - z^2/d)^(k + 1), here with k = (d - 3) / 2.
+double sphere_cell_mean(const Sphere& sp, double lo, double hi) {
+  const double d = sp.d, r = std::sqrt(d);
+  auto g = [&](double z) { return std::fabs(z) >= r ? 0.0 : sphere_power(z, sp.d, (d - 1) / 2); };
+  return sp.c * d / (d - 1) * (g(lo) - g(hi)) / sphere_mass(sp, lo, hi);
+}
+
+// Lloyd's iteration from `lv` (levels ascending) with the given cell-mean rule.
+template <typename CellMean>
+bool lloyd_iterate(int levels, double* lv, CellMean cell_mean) {
+  double next[16], edge[17];
   for (int iter = 0; iter < 1000000; ++iter) {
     edge[0] = -INFINITY;
     edge[levels] = INFINITY;
     for (int j = 1; j < levels; ++j) edge[j] = 0.5 * (lv[j - 1] + lv[j]);
     double moved = 0.0;
     for (int j = 0; j < levels; ++j) {
-      next[j] = (normal_density(edge[j]) - normal_density(edge[j + 1])) /
-                normal_mass(edge[j], edge[j + 1]);
+      next[j] = cell_mean(edge[j], edge[j + 1]);
       moved = std::fmax(moved, std::fabs(next[j] - lv[j]));
     }
     std::memcpy(lv, next, sizeof(double) * levels);
-    if (moved < 1e-14) {
-      std::memcpy(level_out, lv, sizeof(double) * levels);
-      return true;
-    }
+    if (moved < 1e-14) return true;
   }
   return false;
 }
 
+// Levels of the Lloyd-Max quantizer of N(0,1) (kind 0) or of the rotated-
+// coordinate distribution for head_dim d (kind 1, started from the N(0,1)
+// solution).
+bool lloyd_max(int levels, int kind, int d, double* lv) {
+  for (int j = 0; j < levels; ++j) lv[j] = -2.0 + 4.0 * (j + 0.5) / levels;
+  if (!lloyd_iterate(levels, lv, normal_cell_mean)) return false;
+  if (kind == 0) return true;
+  const Sphere sp{d, std::exp(std::lgamma(d / 2.0) - std::lgamma((d - 1) / 2.0)) /
+                         std::sqrt(M_PI * d)};
+  return lloyd_iterate(levels, lv, [&](double lo, double hi) { return sphere_cell_mean(sp, lo, hi); });
+}
+
 // float32 table: odd-symmetric levels, boundaries = float32 midpoints.
-bool build_codebook(int bits, float* cent, float* bnd) {
+bool build_codebook(int bits, int kind, int d, float* cent, float* bnd) {
   const int levels = 1 << bits, half = levels / 2;
   double lv[16];
-  if (!lloyd_max(levels, lv)) return false;
+  if (!lloyd_max(levels, kind, d, lv)) return false;
   for (int j = 0; j < half; ++j) {
     const float pos = (float)((lv[half + j] - lv[half - 1 - j]) / 2.0);
     cent[half + j] = pos;
@@ -121,6 +211,9 @@ tq_status check_params(const tq_params* p) {
     return fail(TQ_ERR_INVALID, "k_bits=%d v_bits=%d: each must be 2, 3 or 4", p->k_bits,
                 p->v_bits);
   if (p->qjl != 0 && p->qjl != 1) return fail(TQ_ERR_INVALID, "qjl must be 0 or 1");
+  if (p->codebook != TQ_CODEBOOK_GAUSSIAN && p->codebook != TQ_CODEBOOK_SPHERE)
+    return fail(TQ_ERR_INVALID, "codebook %d: must be TQ_CODEBOOK_GAUSSIAN or TQ_CODEBOOK_SPHERE",
+                p->codebook);
   return TQ_OK;
 }
 
@@ -201,8 +294,9 @@ tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout
   t.k_bits = params->k_bits;
   t.v_bits = params->v_bits;
   t.qjl = params->qjl;
-  if (!build_codebook(params->k_bits, t.k_cent, t.k_bnd) ||
-      !build_codebook(params->v_bits, t.v_cent, t.v_bnd)) {
+  const int kind = params->codebook, d = params->head_dim;
+  if (!build_codebook(params->k_bits, kind, d, t.k_cent, t.k_bnd) ||
+      !build_codebook(params->v_bits, kind, d, t.v_cent, t.v_bnd)) {
     delete cb;
     return fail(TQ_ERR_INVALID, "Lloyd-Max iteration did not converge");
   }

@@ -34,7 +34,10 @@ EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append", "tq_q
 
 class tq_params(C.Structure):
     _fields_ = [("head_dim", C.c_int), ("k_bits", C.c_int), ("v_bits", C.c_int),
-                ("qjl", C.c_int), ("seed", C.c_uint64)]
+                ("qjl", C.c_int), ("seed", C.c_uint64), ("codebook", C.c_int)]
+
+
+CODEBOOKS = {"gaussian": 0, "sphere": 1}   # TQ_CODEBOOK_GAUSSIAN, TQ_CODEBOOK_SPHERE
 
 
 class tq_layout(C.Structure):
@@ -103,8 +106,14 @@ def kv_bits_split(kv_bits: float) -> tuple[int, int]:
 class Codebook:
     """Owner of a tq_codebook handle (host memory; freed with tq_free)."""
 
-    def __init__(self, head_dim: int, k_bits: int, v_bits: int, qjl: bool = False, seed: int = 0):
-        self.params = tq_params(head_dim, k_bits, v_bits, int(bool(qjl)), seed & ((1 << 64) - 1))
+    def __init__(self, head_dim: int, k_bits: int, v_bits: int, qjl: bool = False, seed: int = 0,
+                 codebook: str = "gaussian"):
+        """codebook: "gaussian" (Lloyd-Max for N(0,1)) or "sphere" (Lloyd-Max for
+        the exact distribution of a rotated coordinate, which depends on head_dim)."""
+        if codebook not in CODEBOOKS:
+            raise ValueError(f"codebook must be one of {sorted(CODEBOOKS)}")
+        self.params = tq_params(head_dim, k_bits, v_bits, int(bool(qjl)), seed & ((1 << 64) - 1),
+                                CODEBOOKS[codebook])
         self.layout = tq_layout()
         h = C.c_void_p()
         _check(lib.tq_codebook_init(C.byref(self.params), C.byref(h), C.byref(self.layout)),
@@ -112,9 +121,10 @@ class Codebook:
         self.handle = h
 
     @classmethod
-    def from_kv_bits(cls, head_dim: int, kv_bits: float, qjl: bool = False, seed: int = 0):
+    def from_kv_bits(cls, head_dim: int, kv_bits: float, qjl: bool = False, seed: int = 0,
+                     codebook: str = "gaussian"):
         kb, vb = kv_bits_split(kv_bits)
-        return cls(head_dim, kb, vb, qjl, seed)
+        return cls(head_dim, kb, vb, qjl, seed, codebook)
 
     head_dim = property(lambda self: self.params.head_dim)
     k_bits = property(lambda self: self.params.k_bits)
