@@ -72,7 +72,7 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 #define TQ_CODEBOOK_SPHERE 1
 
 /* Codec parameters.
- *   head_dim : d, 128 or 256 (64 is reported as TQ_ERR_UNSUPPORTED)
+ *   head_dim : d, 64, 128 or 256
  *   k_bits, v_bits : code widths in {2, 3, 4} ("3.5 bits" = 3 and 4)
  *   qjl      : 1 = keys also carry the 1-bit QJL residual sketch
  *   seed     : seeds the sign vectors of R (and of R2 = RHT2 for QJL).  One R

@@ -74,10 +74,10 @@ def test_codebook_rejects_bad_params(bad):
     assert tq.tq_last_error()
 
 
-def test_head_dim_64_reported_unsupported():
-    params = tq.tq_params(64, 3, 4, 0, 0)
-    h = C.c_void_p()
-    assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_ERR_UNSUPPORTED
+def test_head_dim_64_layout():
+    cb = tq.Codebook(64, 3, 4, qjl=True)
+    assert (cb.layout.k_code_bytes, cb.layout.v_code_bytes, cb.layout.k_sign_bytes) == (24, 32, 8)
+    assert tq.Codebook(64, 3, 4, codebook="sphere").tables()["k_centroids"].shape[0] == 8
 
 
 def _fake_cache(batch=2, kv_heads=2, capacity=64, qjl=False, **over):

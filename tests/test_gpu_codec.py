@@ -43,7 +43,7 @@ def _check_unit(cache, tb, b, h, k_all, v_all, qjl):
 # count (keys and values of every row): up to 4096 vectors one vector per warp,
 # above that 32 channels per lane.  n = 37 and n = 700 (with B = 2, H = 3) fall
 # on either side, so every case runs through both.
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kb,vb", [(2, 2), (2, 3), (3, 3), (3, 4), (4, 4)])
 @pytest.mark.parametrize("qjl", [False, True])
 @pytest.mark.parametrize("n", [37, 700])

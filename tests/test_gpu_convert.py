@@ -36,7 +36,7 @@ def _check_rows(cache, tb, k, v, lengths, qjl, rows=None):
 
 
 @pytest.mark.parametrize("d,kb,vb,qjl", [(128, 3, 4, False), (128, 3, 4, True), (256, 2, 2, True),
-                                         (128, 4, 4, False)])
+                                         (128, 4, 4, False), (64, 3, 4, True)])
 @pytest.mark.parametrize("T,heads_last", [(40, False), (600, False), (600, True)])
 def test_convert_ragged_bit_exact(d, kb, vb, qjl, T, heads_last):
     B, H = 3, 4

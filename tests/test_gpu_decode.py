@@ -56,9 +56,9 @@ def _oracle(d, kb, vb, qjl, seed, k, v, q, lengths, G, scale=None):
     return out
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kb,vb,qjl", [(3, 4, False), (3, 4, True), (2, 2, True), (4, 4, False),
-                                       (2, 3, False), (3, 3, True)])
+                                       (2, 3, False), (3, 3, True), (2, 2, False), (3, 3, False)])
 def test_decode_matches_oracle(d, kb, vb, qjl):
     G, B, Hkv = 4, 2, 2
     lengths = [300, 129]
@@ -66,6 +66,18 @@ def test_decode_matches_oracle(d, kb, vb, qjl):
     out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=320)
     torch.cuda.synchronize()
     ref = _oracle(d, kb, vb, qjl, kb * 10 + vb, k, v, q, lengths, G)
+    assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
+
+
+@pytest.mark.parametrize("G", [1, 8])
+@pytest.mark.parametrize("qjl", [False, True])
+def test_gqa_groups_head_dim_64(G, qjl):
+    d, B, Hkv = 64, 2, 2
+    lengths = [517, 64]
+    cb, cache, k, v, q = _setup(d, 3, 4, qjl, B, Hkv, G, lengths, 528, seed=40 + G, corr=True)
+    out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=528)
+    torch.cuda.synchronize()
+    ref = _oracle(d, 3, 4, qjl, 40 + G, k, v, q, lengths, G)
     assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
 
 

@@ -204,9 +204,8 @@ void build_signs(uint64_t state, int d, uint32_t* mask) {
 
 tq_status check_params(const tq_params* p) {
   if (!p) return fail(TQ_ERR_INVALID, "params is NULL");
-  if (p->head_dim != 128 && p->head_dim != 256)
-    return fail(p->head_dim == 64 ? TQ_ERR_UNSUPPORTED : TQ_ERR_INVALID,
-                "head_dim %d: supported values are 128 and 256", p->head_dim);
+  if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256)
+    return fail(TQ_ERR_INVALID, "head_dim %d: supported values are 64, 128 and 256", p->head_dim);
   if (p->k_bits < 2 || p->k_bits > 4 || p->v_bits < 2 || p->v_bits > 4)
     return fail(TQ_ERR_INVALID, "k_bits=%d v_bits=%d: each must be 2, 3 or 4", p->k_bits,
                 p->v_bits);

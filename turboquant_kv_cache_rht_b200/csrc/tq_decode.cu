@@ -7,6 +7,26 @@ namespace tq {
 
 namespace {
 
+// A lane's E = d/32 consecutive floats of a partial (16- or 8-byte loads).
+template <int E>
+__device__ __forceinline__ void load_lane(const float* p, float (&v)[E]) {
+  if constexpr (E % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < E / 4; ++i) {
+      const float4 x = reinterpret_cast<const float4*>(p)[i];
+      v[4 * i] = x.x;
+      v[4 * i + 1] = x.y;
+      v[4 * i + 2] = x.z;
+      v[4 * i + 3] = x.w;
+    }
+  } else {
+    static_assert(E == 2, "d of 64, 128 or 256");
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x;
+    v[1] = x.y;
+  }
+}
+
 constexpr int kCombineThreads = 256;
 constexpr int kMaxParts = 1024;  // partials one unit can have (at most one per CTA)
 static_assert(kMaxTargetCtas <= kMaxParts, "a unit's partials must fit the merge");
@@ -80,15 +100,11 @@ __global__ void __launch_bounds__(kCombineThreads)
   const float* po = ws + (first * G + hg) * D;              // partial s at po + s * G * D
   const float* pml = ws + (long)nslots * G * D + (first * G + hg) * 2;  // at pml + s * G * 2
   // issue the loads of the first round before anything depends on them
-  float4 ov[PER][E / 4];
+  float ov[PER][E];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int s = warp + W * i;
-    if (s < S) {
-#pragma unroll
-      for (int v = 0; v < E / 4; ++v)
-        ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * G * D + lane * E)[v];
-    }
+    if (s < S) load_lane<E>(po + (long)s * G * D + lane * E, ov[i]);
   }
   float ms[kMaxParts / kCombineThreads], ls[kMaxParts / kCombineThreads];
 #pragma unroll
@@ -137,11 +153,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int s = s0 + warp + W * i;
-        if (s < S) {
-#pragma unroll
-          for (int v = 0; v < E / 4; ++v)
-            ov[i][v] = reinterpret_cast<const float4*>(po + (long)s * G * D + lane * E)[v];
-        }
+        if (s < S) load_lane<E>(po + (long)s * G * D + lane * E, ov[i]);
       }
     }
 #pragma unroll
@@ -151,12 +163,7 @@ __global__ void __launch_bounds__(kCombineThreads)
         const float w = wgt[s];
         if (w > 0.f) {  // skips the slots no CTA wrote
 #pragma unroll
-          for (int v = 0; v < E / 4; ++v) {
-            a[4 * v] = fmaf(ov[i][v].x, w, a[4 * v]);
-            a[4 * v + 1] = fmaf(ov[i][v].y, w, a[4 * v + 1]);
-            a[4 * v + 2] = fmaf(ov[i][v].z, w, a[4 * v + 2]);
-            a[4 * v + 3] = fmaf(ov[i][v].w, w, a[4 * v + 3]);
-          }
+          for (int e = 0; e < E; ++e) a[e] = fmaf(ov[i][e], w, a[e]);
         }
       }
     }
@@ -203,7 +210,7 @@ size_t decode_workspace_bytes(const DecodePlan& plan, int q_heads, int kv_heads,
 
 bool decode_supported(int head_dim, int group, int k_bits, int v_bits, int qjl) {
   (void)qjl;
-  if (head_dim != 128 && head_dim != 256) return false;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return false;
   if (group != 1 && group != 2 && group != 4 && group != 8) return false;
   if (k_bits < 2 || k_bits > 4) return false;
   return v_bits == k_bits || v_bits == k_bits + 1;
@@ -220,12 +227,15 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = tb.d == 128 ? decode_occupancy_dim<128>(tb, group, &ctas_per_sm)
-                  : decode_occupancy_dim<256>(tb, group, &ctas_per_sm);
+  e = tb.d == 64    ? decode_occupancy_dim<64>(tb, group, &ctas_per_sm)
+      : tb.d == 128 ? decode_occupancy_dim<128>(tb, group, &ctas_per_sm)
+                    : decode_occupancy_dim<256>(tb, group, &ctas_per_sm);
   if (e != cudaSuccess) return e;
   const long target = std::min<long>(kMaxTargetCtas, (long)std::max(ctas_per_sm, 1) * sms);
   const DecodePlan plan = plan_decode(cv.batch, cv.kv_heads, max_ctx, target);
-  if (tb.d == 128)
+  if (tb.d == 64)
+    e = launch_decode_dim<64>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+  else if (tb.d == 128)
     e = launch_decode_dim<128>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
   else if (tb.d == 256)
     e = launch_decode_dim<256>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
@@ -241,7 +251,10 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (tb.d == 128)
+  if (tb.d == 64)
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<64>, tb, cv, (const float*)workspace, q_heads,
+                           max_ctx, plan.ctas, plan.slots, out);
+  else if (tb.d == 128)
     e = cudaLaunchKernelEx(&cfg, combine_kernel<128>, tb, cv, (const float*)workspace, q_heads,
                            max_ctx, plan.ctas, plan.slots, out);
   else

@@ -55,6 +55,17 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
 }
+// 8-byte form, for rows whose length is not a multiple of 16 bytes (d = 64
+// with 3-bit codes); both addresses are 8-byte aligned.
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+template <int CB>
+__device__ __forceinline__ void cp_async_chunk(void* smem, const void* gmem) {
+  if constexpr (CB == 16) cp_async16(smem, gmem);
+  else cp_async8(smem, gmem);
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
@@ -149,7 +160,8 @@ __device__ __forceinline__ void warp_fwht(float (&u)[E], int lane) {
 // pattern allows); multiples of 4 words for 16-byte copies.
 constexpr int k_stride_words(int d, int bits) { return (d == 256 && bits == 4) ? 36 : bits * d / 32; }
 constexpr int v_stride_words(int d, int bits) {
-  return d == 128 ? (bits == 4 ? 20 : 12) : (bits == 2 ? 20 : bits == 3 ? 28 : 36);
+  return d == 64 ? (bits == 2 ? 4 : 12)
+                 : d == 128 ? (bits == 4 ? 20 : 12) : (bits == 2 ? 20 : bits == 3 ? 28 : 36);
 }
 
 template <int D, int G, int KB, int VB, bool QJL>
@@ -163,8 +175,12 @@ struct DecodeGeom {
   static constexpr int KS = k_stride_words(D, KB);
   static constexpr int VS = v_stride_words(D, VB);
   static constexpr int SS = D / 32;
-  static constexpr int KW = KB * D / 128;     // key words per thread quarter
-  static constexpr int SW = D / 128;          // sign words per thread quarter
+  static constexpr int QB = KB * D / 4;       // key bits per thread quarter (a slice of the row)
+  static constexpr int KW = (QB + 31) / 32;   // words of the slice, aligned to bit 0
+  static constexpr int KNW = (QB % 32 == 0) ? QB / 32 : (QB + 16 + 31) / 32;  // words it spans
+  static constexpr int SW = D >= 128 ? D / 128 : 1;  // sign words per thread quarter (d = 64: half a word)
+  static constexpr int CBK = (kRowB % 16 == 0) ? 16 : 8;  // copy chunk bytes per row
+  static constexpr int CBV = (vRowB % 16 == 0) ? 16 : 8;
   static constexpr int VCH = VB * D / 8;      // value bits per thread group
   static constexpr int VCW = (VCH + 31) / 32; // words of the aligned value chunk
   static constexpr int VNW = (VCH % 32 == 0) ? VCH / 32 : (VCH + 16 + 31) / 32;
@@ -201,7 +217,7 @@ struct DecodeGeom {
   static constexpr int offSched = (offRed + redFloats * 4 + 15) / 16 * 16;
   static constexpr int schedBytes = kDecWarps * 8 + kDecThreads * 4 + kDecThreads * 8;
   static constexpr int total = offSched + schedBytes;
-  static_assert((KS % 4) == 0 && (VS % 4) == 0, "16-byte aligned rows");
+  static_assert((KS * 4) % CBK == 0 && (VS * 4) % CBV == 0, "rows aligned to the copy chunk");
   static_assert(VCW <= 4 && VNW <= 4, "value chunk too wide");
 };
 
@@ -313,11 +329,11 @@ __device__ __forceinline__ long long block_exclusive_scan(long long x, long long
   return before + inc - x;
 }
 
-// CTAs per SM the register budget is sized for: d = 128 fits four CTAs (128
+// CTAs per SM the register budget is sized for: d <= 128 fits four CTAs (128
 // registers) unless the shape carries two column tiles or the QJL sketch,
 // which need up to 168 registers (three CTAs); d = 256 fits two.
 template <int D, int G, bool QJL>
-constexpr int decode_min_ctas() { return D == 128 ? ((G > 4 || QJL) ? 3 : 4) : 2; }
+constexpr int decode_min_ctas() { return D <= 128 ? ((G > 4 || QJL) ? 3 : 4) : 2; }
 
 template <int D, int G, int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
@@ -391,30 +407,31 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 
   // This thread's share of every tile copy: the chunk offsets are the same for
   // all tiles, so they are computed once (stage offset and tile base vary).
-  constexpr int CK = Geo::kRowB / 16, CV = Geo::vRowB / 16, CS = Geo::sRowB / 16;
+  constexpr int CK = Geo::kRowB / Geo::CBK, CV = Geo::vRowB / Geo::CBV;
+  constexpr int SCH = kDecTile * Geo::sRowB / 16;  // 16-byte chunks of a tile's sign rows (unpadded)
   constexpr int NK = (kDecTile * CK + kDecThreads - 1) / kDecThreads;
   constexpr int NV = (kDecTile * CV + kDecThreads - 1) / kDecThreads;
-  constexpr int NS = QJL ? (kDecTile * CS + kDecThreads - 1) / kDecThreads : 0;
+  constexpr int NS = QJL ? (SCH + kDecThreads - 1) / kDecThreads : 0;
   int k_dst[NK], k_src[NK], k_row[NK], v_dst[NV], v_src[NV], v_row[NV];
   int s_dst[NS > 0 ? NS : 1], s_row[NS > 0 ? NS : 1];
 #pragma unroll
   for (int i = 0; i < NK; ++i) {
     const int c = tid + kDecThreads * i, r = c / CK, col = c - r * CK;
     k_row[i] = c < kDecTile * CK ? r : kDecTile;
-    k_dst[i] = Geo::offK + r * Geo::KS * 4 + col * 16;
-    k_src[i] = r * Geo::kRowB + col * 16;
+    k_dst[i] = Geo::offK + r * Geo::KS * 4 + col * Geo::CBK;
+    k_src[i] = r * Geo::kRowB + col * Geo::CBK;
   }
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = tid + kDecThreads * i, r = c / CV, col = c - r * CV;
     v_row[i] = c < kDecTile * CV ? r : kDecTile;
-    v_dst[i] = Geo::offV + r * Geo::VS * 4 + col * 16;
-    v_src[i] = r * Geo::vRowB + col * 16;
+    v_dst[i] = Geo::offV + r * Geo::VS * 4 + col * Geo::CBV;
+    v_src[i] = r * Geo::vRowB + col * Geo::CBV;
   }
 #pragma unroll
   for (int i = 0; i < NS; ++i) {
     const int c = tid + kDecThreads * i;
-    s_row[i] = c < kDecTile * CS ? c / CS : kDecTile;
+    s_row[i] = c < SCH ? c * 16 / Geo::sRowB : kDecTile;  // first row the chunk holds
     s_dst[i] = Geo::offS + c * 16;
   }
   auto issue_tile = [&](int stage, int start) {
@@ -425,10 +442,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     const uint8_t* vb = cv.v_codes + (row_slot + start) * Geo::vRowB;
 #pragma unroll
     for (int i = 0; i < NK; ++i)
-      if (k_row[i] < rows) cp_async16(st + k_dst[i], kb + k_src[i]);
+      if (k_row[i] < rows) cp_async_chunk<Geo::CBK>(st + k_dst[i], kb + k_src[i]);
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-      if (v_row[i] < rows) cp_async16(st + v_dst[i], vb + v_src[i]);
+      if (v_row[i] < rows) cp_async_chunk<Geo::CBV>(st + v_dst[i], vb + v_src[i]);
     if constexpr (QJL) {
       const uint8_t* sb = cv.k_signs + (row_slot + start) * Geo::sRowB;
 #pragma unroll
@@ -532,12 +549,15 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       bk[j][kb][0] = live ? (part ? l01 : h01) : 0u;
       bk[j][kb][1] = live ? (part ? l23 : h23) : 0u;
       if constexpr (QJL) {
-        // sign slots 2q,2q+1 -> bits (j0, j0+16) of word kb/8; 2q+8,2q+9 -> (j0+8, j0+24)
-        const int base = qd * (D / 4) + 32 * (kb >> 3) + (kb & 7);
+        // d >= 128: sign slots 2q,2q+1 -> bits (j0, j0+16) of word kb/8 of the
+        // quarter, 2q+8,2q+9 -> (j0+8, j0+24).  d = 64 (16 bits per quarter):
+        // slots 2q,2q+1 -> bits (kb, kb+8), 2q+8,2q+9 -> (kb+4, kb+12).
+        const int base = D >= 128 ? qd * (D / 4) + 32 * (kb >> 3) + (kb & 7) : qd * 16 + kb;
+        constexpr int P1 = D >= 128 ? 16 : 8, P2 = D >= 128 ? 8 : 4, P3 = D >= 128 ? 24 : 12;
         const float* r2 = qs2 + (live ? head : 0) * D;
         uint32_t a_h, a_l, b_h, b_l;
-        split_pair(r2[base] * qsc2, r2[base + 16] * qsc2, a_h, a_l);
-        split_pair(r2[base + 8] * qsc2, r2[base + 24] * qsc2, b_h, b_l);
+        split_pair(r2[base] * qsc2, r2[base + P1] * qsc2, a_h, a_l);
+        split_pair(r2[base + P2] * qsc2, r2[base + P3] * qsc2, b_h, b_l);
         bq[j][kb][0] = live ? (part ? a_l : a_h) : 0u;
         bq[j][kb][1] = live ? (part ? b_l : b_h) : 0u;
       }
@@ -623,12 +643,9 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
         for (int e = 0; e < 4; ++e) sacc[par][j][e] = sacc2[par][j][e] = 0.f;
     {
       uint32_t kw0[Geo::KW], kw1[Geo::KW];
-      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS + qd * Geo::KW;
-#pragma unroll
-      for (int w = 0; w < Geo::KW; ++w) {
-        kw0[w] = k0[w];
-        kw1[w] = k0[8 * Geo::KS + w];
-      }
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
+      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);  // bits of quarter qd, tokens g
+      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);  // and g + 8
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
@@ -662,17 +679,27 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
         for (int j = 0; j < NT; ++j) qacc[par][j][0] = qacc[par][j][1] = qacc[par][j][2] = qacc[par][j][3] = 0.f;
       uint32_t sw0[Geo::SW], sw1[Geo::SW];
-      const uint32_t* s0p = reinterpret_cast<const uint32_t*>(st + Geo::offS) + (r0 + g) * Geo::SS + qd * Geo::SW;
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(st + Geo::offS) + (r0 + g) * Geo::SS;
+      if constexpr (D >= 128) {
 #pragma unroll
-      for (int w = 0; w < Geo::SW; ++w) {
-        sw0[w] = s0p[w];
-        sw1[w] = s0p[8 * Geo::SS + w];
+        for (int w = 0; w < Geo::SW; ++w) {
+          sw0[w] = srow[qd * Geo::SW + w];
+          sw1[w] = srow[8 * Geo::SS + qd * Geo::SW + w];
+        }
+      } else {
+        // the quarter's 16 bits h, with a copy shifted up by 8: then bit 15 and
+        // bit 31 of (x << (15 - kb)) are h[kb] and h[kb + 8]
+        const int sh = 16 * (qd & 1);
+        const uint32_t h0 = (srow[qd >> 1] >> sh) & 0xffffu, h1 = (srow[8 * Geo::SS + (qd >> 1)] >> sh) & 0xffffu;
+        sw0[0] = h0 | (h0 << 8);
+        sw1[0] = h1 | (h1 << 8);
       }
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
-        const int wi = kb >> 3, j0 = kb & 7;
+        const int wi = D >= 128 ? kb >> 3 : 0, j0 = D >= 128 ? kb & 7 : kb;
+        constexpr int S2 = D >= 128 ? 7 : 11;  // shift that brings the second pair to bits 15, 31
         const uint32_t a0 = sign_pair(sw0[wi] << (15 - j0)), a1 = sign_pair(sw1[wi] << (15 - j0));
-        const uint32_t a2 = sign_pair(sw0[wi] << (7 - j0)), a3 = sign_pair(sw1[wi] << (7 - j0));
+        const uint32_t a2 = sign_pair(sw0[wi] << (S2 - j0)), a3 = sign_pair(sw1[wi] << (S2 - j0));
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma16816(qacc[kb & 1][j], a0, a1, a2, a3, bq[j][kb][0], bq[j][kb][1]);
       }

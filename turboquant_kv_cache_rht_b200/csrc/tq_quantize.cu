@@ -34,9 +34,9 @@ constexpr int kAppendWarps = 8;
 constexpr int kAppendThreads = 32 * kAppendWarps;
 constexpr unsigned kFull = 0xffffffffu;
 
-// The lane's E consecutive input elements as fp32, read as 16- or 8-byte
-// words (the row start is 16-byte aligned because k and v are, and E
-// elements of any input type span a multiple of 8 bytes).
+// The lane's E consecutive input elements as fp32, read as 16-, 8- or 4-byte
+// words (the row start is 16-byte aligned because k and v are, and the E
+// elements of a lane span a multiple of that word).
 template <int E, typename T>
 __device__ __forceinline__ void load_elems(const T* p, float (&x)[E]) {
   constexpr int NB = E * (int)sizeof(T), NW = NB / 4;
@@ -50,11 +50,13 @@ __device__ __forceinline__ void load_elems(const T* p, float (&x)[E]) {
       w[4 * i + 2] = v.z;
       w[4 * i + 3] = v.w;
     }
-  } else {
-    static_assert(NB == 8, "8 or a multiple of 16 bytes per lane");
+  } else if constexpr (NB == 8) {
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
     w[0] = v.x;
     w[1] = v.y;
+  } else {
+    static_assert(NB == 4, "4, 8 or a multiple of 16 bytes per lane");
+    w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
   }
 #pragma unroll
   for (int i = 0; i < NW; ++i) {
@@ -470,6 +472,7 @@ cudaError_t launch_dim(const Tables& tb, const CacheView& cv, const void* k, con
 cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const void* k,
                                    const void* v, int dtype, int n_new, cudaStream_t stream) {
   switch (tb.d) {
+    case 64: return launch_dim<64>(tb, cv, k, v, dtype, n_new, stream);
     case 128: return launch_dim<128>(tb, cv, k, v, dtype, n_new, stream);
     case 256: return launch_dim<256>(tb, cv, k, v, dtype, n_new, stream);
   }
@@ -481,6 +484,9 @@ cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const v
                                   long stride_t, const int32_t* lengths, int max_len,
                                   cudaStream_t stream) {
   switch (tb.d) {
+    case 64:
+      return launch_convert_dim<64>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                    max_len, stream);
     case 128:
       return launch_convert_dim<128>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
                                      max_len, stream);
