@@ -54,10 +54,10 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d128.cu", "tq_decode_d256.cu",
                   "tq_internal.cuh")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31746048, "c127026c84fdb290"),
-    "qjl": (566686976, "c127026c84fdb290"),
-    "long": (352887808, "c127026c84fdb290"),
-    "serving": (1102792192, "c127026c84fdb290"),
+    "gqa": (31748096, "41795a16fa794c1b"),
+    "qjl": (566693888, "41795a16fa794c1b"),
+    "long": (353863168, "41795a16fa794c1b"),
+    "serving": (1102753280, "41795a16fa794c1b"),
 }
 
 
