@@ -450,6 +450,39 @@ def dense_attention(q: np.ndarray, keys: np.ndarray, vals: np.ndarray,
     return (p @ vals) / p.sum(axis=-1, keepdims=True)
 
 
+# ---------------------------------------------------------------------------
+# Weights regime ([P3] introduction: "Weights (MSE regime)": rotate each weight
+# matrix, then quantize; "The Metal kernels" item 1: a non-uniform LUT dequant
+# + matmul computed directly on packed indices).  Reading: each row of
+# W [N][K] is cut into K/d blocks of d input channels, and every block is
+# encoded exactly as a KV vector is (fp16 norm, rotation, Lloyd-Max codes).
+# ---------------------------------------------------------------------------
+def weights_encode(w: np.ndarray, s1: np.ndarray, centroids: np.ndarray,
+                   boundaries: np.ndarray, bits: int) -> dict:
+    """w float32 [N][K] -> idx [K/d][N][d], codes [K/d][N][bits*d/8], norm16 [K/d][N]
+    (block j of every row is encoded by ``encode``; d = len(s1))."""
+    w = np.asarray(w, np.float32)
+    d = len(s1)
+    n, k = w.shape
+    blocks = w.reshape(n, k // d, d).transpose(1, 0, 2)
+    enc = [encode(blocks[j], s1, centroids, boundaries, bits) for j in range(k // d)]
+    return {key: np.stack([e[key] for e in enc]) for key in ("idx", "codes", "norm16")}
+
+
+def weights_dequantize(idx: np.ndarray, norm16: np.ndarray, s1: np.ndarray,
+                       centroids: np.ndarray) -> np.ndarray:
+    """W_hat float64 [N][K]: block j of row n is R^T (n16 c[idx] / sqrt(d))."""
+    blocks = [rht_inverse(dequantize_rotated(idx[j], norm16[j], centroids), s1)
+              for j in range(idx.shape[0])]
+    return np.concatenate(blocks, axis=1)
+
+
+def lut_matmul(x: np.ndarray, idx: np.ndarray, norm16: np.ndarray, s1: np.ndarray,
+               centroids: np.ndarray) -> np.ndarray:
+    """Y = X W_hat^T in float64 for X [M][K]."""
+    return np.asarray(x, np.float64) @ weights_dequantize(idx, norm16, s1, centroids).T
+
+
 def kv_bits_split(kv_bits: float) -> tuple[int, int]:
     """Key and value bit widths for a (possibly fractional) kv_bits.
 
