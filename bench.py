@@ -1,7 +1,7 @@
 """Benchmark of the TurboQuant decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa|qjl|long|serving|tiny]
-                    [--impl ours|reference] [--no-dense] [--no-cpu-baseline]
+                    [--impl ours|reference] [--no-dense] [--no-cpu-baseline] [--lutmm]
 
 A step is one pass of the whole hot path over one batch: tq_quantize_append of
 one new token per (batch row, KV head), then tq_decode_attention of every query
@@ -346,6 +346,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     dense = None
     if not args.no_dense and world == 1:
         dense = dense_baselines(w, st, dev)
+    lutmm = lut_matmul_bench(dev, peaks()[0]) if (args.lutmm and world == 1) else None
 
     del graphs
     peak, peak_kind = peaks()
@@ -383,6 +384,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     }
     if dense is not None:
         res["dense_baseline"] = dense
+    if lutmm is not None:
+        res["lut_matmul"] = lutmm
     return res
 
 
@@ -446,6 +449,52 @@ def end_to_end(st: State, dev, K: int, stream) -> dict:
     d2h = hout.numel() * hout.element_size()
     return {"value": round(byts / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms / K, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def lut_matmul_bench(dev, peak_gbs: float, rows: int = 16384, k: int = 8192, bits: int = 4,
+                     head_dim: int = 128, replicas: int = 8) -> dict:
+    """The weights-regime LUT matmul on a synthetic [rows, k] layer (seeded N(0,1)
+    weights): packed bytes per call over the back-to-back call time, for 1 and 16
+    inputs, beside torch's dense bf16 product with the same weights.  The codes are
+    replicated (replicas x codes > 4x L2) and calls rotate over them."""
+    from turboquant_kv_cache_rht_b200 import tq
+    g = torch.Generator(device=dev).manual_seed(20250)
+    wt = torch.randn(rows, k, generator=g, device=dev).bfloat16()
+    cb = tq.Codebook(head_dim, bits, bits, seed=5)
+    qw = tq.QuantizedWeights(cb, wt)
+    copies = [qw]
+    for _ in range(replicas - 1):
+        c = tq.QuantizedWeights.__new__(tq.QuantizedWeights)
+        c.cb, c.rows, c.k = cb, rows, k
+        c.codes, c.norms = qw.codes.clone(), qw.norms.clone()
+        copies.append(c)
+    packed = qw.codes.numel() + qw.norms.numel() * 2
+
+    def timed(fn, n):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize(dev)
+        torch.cuda._sleep(1_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return 1e3 * e0.elapsed_time(e1) / n
+
+    res = {"shape": [rows, k], "bits": bits, "head_dim": head_dim, "packed_bytes": packed}
+    dense_w = [wt] + [wt.clone() for _ in range(2)]   # 3 x 256 MB bf16 copies, > 4x L2
+    for m in (1, 16):
+        x = torch.randn(m, k, generator=g, device=dev).bfloat16()
+        us = timed(lambda i: copies[i % replicas].matmul(x), 4 * replicas)
+        dus = timed(lambda i: torch.matmul(x, dense_w[i % 3].T), 12)
+        gbs = (packed + x.numel() * 2 + m * rows * 4) / (us * 1e-6) / 1e9
+        res[f"m{m}"] = {"us": round(us, 2), "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak_gbs, 4),
+                        "dense_bf16_us": round(dus, 2), "speedup_vs_dense": round(dus / us, 2)}
+    del copies, dense_w, wt
+    torch.cuda.empty_cache()
+    return res
 
 
 def dense_baselines(w: wl.Workload, st: State, dev) -> dict:
@@ -628,6 +677,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lutmm", action="store_true",
+                    help="also time the weights-regime LUT matmul on a 16384 x 8192 layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

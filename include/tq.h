@@ -235,6 +235,37 @@ tq_status tq_decode_attention_noalloc(const tq_codebook* cb, const tq_cache* cac
                                       tq_dtype dtype, int q_heads, float softmax_scale,
                                       int max_ctx, float* out, void* stream);
 
+/* Weights regime ("mlx-turboquant" README, introduction: "Weights (MSE
+ * regime)", rotate each weight matrix, then quantize; "The Metal kernels"
+ * item 1: LUT dequant + matmul directly on packed indices).  Each row of a
+ * weight matrix W [rows][k] is cut into k / head_dim blocks of head_dim input
+ * channels, and every block is encoded exactly as a key vector is (fp16 norm,
+ * rotation, k_bits Lloyd-Max codes; the codebook's QJL setting is ignored).
+ *
+ * tq_weights_quantize: w DEVICE [rows][k] of `dtype`, 16-byte aligned;
+ *   codes DEVICE uint8 [k / head_dim][rows][k_bits * head_dim / 8];
+ *   norms DEVICE fp16 bits [k / head_dim][rows]; both 16-byte aligned.
+ *   rows must be a multiple of 16 and k a multiple of head_dim. */
+tq_status tq_weights_quantize(const tq_codebook* cb, const void* w, tq_dtype dtype, int rows, int k,
+                              uint8_t* codes, uint16_t* norms, void* stream);
+
+/* Workspace bytes tq_lut_matmul needs for these sizes (0 when it needs none,
+ * or on bad sizes).  The matmul splits the k blocks over CTAs when rows x m
+ * alone give too few, and the workspace holds the per-split partial sums:
+ * splits * m * rows * 4 bytes. */
+size_t tq_lut_matmul_workspace_bytes(const tq_codebook* cb, int rows, int k, int m);
+
+/* Y = X W_hat^T on the codes of tq_weights_quantize, never forming W_hat:
+ *   y[i][n] = sum_j (norm_{n,j} / sqrt(d)) <centroid[codes_{n,j}], R x_{i,j}>
+ * with x_{i,j} block j of input row i and R the codebook's rotation.
+ * x DEVICE [m][k] of `dtype`; y DEVICE float32 [m][rows]; workspace DEVICE of
+ * at least tq_lut_matmul_workspace_bytes (TQ_ERR_CAPACITY otherwise; NULL
+ * when that is 0).  All 16-byte aligned.  The result is deterministic: the
+ * split partials are added in a fixed order. */
+tq_status tq_lut_matmul(const tq_codebook* cb, const uint8_t* codes, const uint16_t* norms, int rows,
+                        int k, const void* x, tq_dtype dtype, int m, float* y, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
 /* Releases a codebook (NULL is ignored). */
 void tq_free(tq_codebook* cb);
 

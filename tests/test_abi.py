@@ -134,6 +134,32 @@ def test_convert_validation():
     assert _convert(cb, _fake_cache(), strides=(-128, 128, 128)) == tq.TQ_ERR_INVALID
 
 
+def test_weights_validation():
+    """Rejected before any launch (fake pointers; no GPU is touched)."""
+    cb = tq.Codebook(128, 4, 4)
+    wq = lambda rows=64, k=512, dtype=1, w=1 << 12, codes=1 << 13, norms=1 << 14: tq.lib.tq_weights_quantize(
+        cb.handle, w, dtype, rows, k, codes, norms, None)
+    assert wq(rows=40) == tq.TQ_ERR_INVALID          # not a multiple of 16
+    assert wq(k=500) == tq.TQ_ERR_INVALID            # not a multiple of head_dim
+    assert wq(dtype=9) == tq.TQ_ERR_INVALID
+    assert wq(w=0) == tq.TQ_ERR_INVALID
+    assert wq(codes=(1 << 13) + 4) == tq.TQ_ERR_INVALID
+    mm = lambda rows=64, k=512, m=1, ws=0, nbytes=0, y=1 << 15: tq.lib.tq_lut_matmul(
+        cb.handle, 1 << 13, 1 << 14, rows, k, 1 << 12, 1, m, y, ws, nbytes, None)
+    assert mm(m=0) == tq.TQ_ERR_INVALID
+    assert mm(y=0) == tq.TQ_ERR_INVALID
+    need = tq.tq_lut_matmul_workspace_bytes(cb, 64, 512, 1)
+    assert need > 0 and mm(ws=1 << 16, nbytes=need - 4) == tq.TQ_ERR_CAPACITY
+    assert tq.tq_lut_matmul_workspace_bytes(cb, 64, 500, 1) == 0       # bad k
+    # rotated inputs: 4 blocks x 1 group of 4 inputs x (8 k-blocks x 32 lanes x 2 words
+    # + 4 scales); 64 rows x 1 group is one tile, so the 4 blocks are split one per
+    # CTA and the partial sums (4 x 1 x 64) follow
+    assert need == (4 * 1 * 8 * 32 * 2 + 4 * 1 * 4 + 4 * 1 * 64) * 4
+    # more 128-row tiles than the 592-CTA bound need no split: rotated inputs only
+    # (8 inputs -> one group of 8)
+    assert tq.tq_lut_matmul_workspace_bytes(cb, 128 * 600, 512, 8) == (4 * 2 * 8 * 64 + 4 * 8) * 4
+
+
 def _decode(cb, cache, q_heads=4, max_ctx=64, ws=1 << 14, ws_bytes=1 << 30, scale=0.0, q=1 << 12):
     return tq.lib.tq_decode_attention(cb.handle, C.byref(cache), q, 1, q_heads, scale, max_ctx,
                                       1 << 13, ws, ws_bytes, None)

@@ -372,6 +372,52 @@ tq_status tq_quantize_cache(const tq_codebook* cb, const tq_cache* cache, const 
                      "quantize-cache launch");
 }
 
+static tq_status check_weights(const tq_codebook* cb, int rows, int k, tq_dtype dtype) {
+  if (!cb) return fail(TQ_ERR_INVALID, "codebook is NULL");
+  if (rows <= 0 || rows % 16) return fail(TQ_ERR_INVALID, "rows %d: a positive multiple of 16", rows);
+  const int d = cb->params.head_dim;
+  if (k <= 0 || k % d) return fail(TQ_ERR_INVALID, "k %d: a positive multiple of head_dim %d", k, d);
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  return TQ_OK;
+}
+
+tq_status tq_weights_quantize(const tq_codebook* cb, const void* w, tq_dtype dtype, int rows, int k,
+                              uint8_t* codes, uint16_t* norms, void* stream) {
+  tq_status st = check_weights(cb, rows, k, dtype);
+  if (st != TQ_OK) return st;
+  if (!w || !codes || !norms) return fail(TQ_ERR_INVALID, "w, codes or norms is NULL");
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(norms))
+    return fail(TQ_ERR_INVALID, "w, codes and norms must be 16-byte aligned");
+  return cuda_status(tq::launch_weights_quantize(cb->tables, w, (int)dtype, rows, k, codes, norms,
+                                                 (cudaStream_t)stream),
+                     "weights-quantize launch");
+}
+
+size_t tq_lut_matmul_workspace_bytes(const tq_codebook* cb, int rows, int k, int m) {
+  if (!cb || rows <= 0 || rows % 16 || k <= 0 || k % cb->params.head_dim || m <= 0) return 0;
+  return tq::lut_matmul_workspace_bytes(tq::plan_lut_matmul(rows, k, m, cb->params.head_dim, tq::kLutMatmulMaxCtas), rows, m);
+}
+
+tq_status tq_lut_matmul(const tq_codebook* cb, const uint8_t* codes, const uint16_t* norms, int rows,
+                        int k, const void* x, tq_dtype dtype, int m, float* y, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  tq_status st = check_weights(cb, rows, k, dtype);
+  if (st != TQ_OK) return st;
+  if (m <= 0 || m > 65535 * 4) return fail(TQ_ERR_INVALID, "m %d out of range", m);
+  if (!codes || !norms || !x || !y) return fail(TQ_ERR_INVALID, "codes, norms, x or y is NULL");
+  if (!aligned16(codes) || !aligned16(norms) || !aligned16(x) || !aligned16(y))
+    return fail(TQ_ERR_INVALID, "codes, norms, x and y must be 16-byte aligned");
+  const size_t need =
+      tq::lut_matmul_workspace_bytes(tq::plan_lut_matmul(rows, k, m, cb->params.head_dim, tq::kLutMatmulMaxCtas), rows, m);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(TQ_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  if (need > 0 && !aligned16(workspace)) return fail(TQ_ERR_INVALID, "workspace must be 16-byte aligned");
+  return cuda_status(tq::launch_lut_matmul(cb->tables, codes, norms, rows, k, x, (int)dtype, m, y,
+                                           (float*)workspace, (cudaStream_t)stream),
+                     "lut-matmul launch");
+}
+
 size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
                                  int max_ctx) {
   if (!cb || batch <= 0 || q_heads <= 0 || kv_heads <= 0 || max_ctx < 0 ||

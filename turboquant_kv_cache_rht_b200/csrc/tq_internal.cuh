@@ -44,6 +44,27 @@ enum DType : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
 cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const void* k,
                                    const void* v, int dtype, int n_new, cudaStream_t stream);
+// Weights [rows][k] -> codes [k/d][rows][k_bits*d/8] and fp16 norms [k/d][rows].
+cudaError_t launch_weights_quantize(const Tables& tb, const void* w, int dtype, int rows, int k,
+                                    uint8_t* codes, uint16_t* norms, cudaStream_t stream);
+// Y [m][rows] = X [m][k] W_hat^T on the codes above; the workspace holds the
+// rotated inputs (B-fragment order, with their scales) and, when the plan
+// splits the blocks, the per-split partial sums.
+struct MatmulPlan {
+  int inputs_per_group;  // inputs per CTA column group (4 or 8)
+  int groups;            // column groups
+  int splits;            // CTAs along the k blocks
+  int blocks_per_split;
+  size_t frag_words;     // rotated-input fragments in the workspace
+  size_t scale_floats;   // and their scales
+};
+// At most target_ctas CTAs (never more than the bound the workspace is sized for).
+MatmulPlan plan_lut_matmul(int rows, int k, int m, int d, long target_ctas);
+constexpr long kLutMatmulMaxCtas = 148L * 4;
+size_t lut_matmul_workspace_bytes(const MatmulPlan& plan, int rows, int m);
+cudaError_t launch_lut_matmul(const Tables& tb, const uint8_t* codes, const uint16_t* norms, int rows,
+                              int k, const void* x, int dtype, int m, float* y, float* workspace,
+                              cudaStream_t stream);
 // Dense cache (strides in elements) -> compressed cache, lengths[b] tokens per row.
 cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const void* k,
                                   const void* v, int dtype, long stride_b, long stride_h,

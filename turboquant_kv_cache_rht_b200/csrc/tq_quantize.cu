@@ -315,10 +315,12 @@ __global__ void __launch_bounds__(kAppendThreads)
   pdl_trigger();
 }
 
-// Conversion of a dense cache.  Grid: (2 * blocks_per_kind, batch) as for the
-// append; the vectors (h, t) of a row are numbered with t outermost when the
-// input's head stride is the smaller one (a [batch][T][heads][d] cache) and
-// with h outermost otherwise, so consecutive lanes read consecutive memory.
+// Conversion of a dense cache.  Grid: (kinds * blocks_per_kind, batch) as for
+// the append (kinds = 1 encodes keys only: weight blocks); the vectors (h, t)
+// of a row are numbered with t outermost when the input's head stride is the
+// smaller one (a [batch][T][heads][d] cache) and with h outermost otherwise,
+// so consecutive lanes read consecutive memory.  Without `lengths` every row
+// holds max_len vectors and no length or flag is written.
 template <int D, typename T, int E>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_convert_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
@@ -340,10 +342,10 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int t = !in_grid ? 0 : heads_inner ? (int)(r / H) : (int)(r % max_len);
 
   pdl_wait();
-  const int asked = max(lengths[b], 0);
+  const int asked = lengths ? max(lengths[b], 0) : max_len;
   const int len = min(asked, max_len);
   const bool fits = len <= cv.capacity;
-  if (tid == 0 && blockIdx.x == 0) {
+  if (tid == 0 && blockIdx.x == 0 && lengths) {
     if (asked > max_len) atomicOr(cv.status, (int)kFlagMaxCtx);
     if (fits) cv.seq_lens[b] = len;  // no block of this grid reads seq_lens
     else atomicOr(cv.status, (int)kFlagCapacity);
@@ -414,13 +416,14 @@ cudaError_t launch_typed(const Tables& tb, const CacheView& cv, const void* k, c
 template <int D, typename T, int E>
 cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const void* k,
                                   const void* v, long sb, long sh, long st,
-                                  const int32_t* lengths, int max_len, cudaStream_t stream) {
+                                  const int32_t* lengths, int max_len, int kinds,
+                                  cudaStream_t stream) {
   constexpr int VPB = kAppendThreads / (D / E);
   const long per_kind = (long)cv.kv_heads * max_len;
   const long blocks_per_kind = std::max<long>(1, (per_kind + VPB - 1) / VPB);
-  if (2 * blocks_per_kind > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
+  if (kinds * blocks_per_kind > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * blocks_per_kind), (unsigned)cv.batch);
+  cfg.gridDim = dim3((unsigned)(kinds * blocks_per_kind), (unsigned)cv.batch);
   cfg.blockDim = dim3(kAppendThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -436,22 +439,26 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
 template <int D, typename T>
 cudaError_t launch_convert_typed(const Tables& tb, const CacheView& cv, const void* k,
                                  const void* v, long sb, long sh, long st, const int32_t* lengths,
-                                 int max_len, cudaStream_t stream) {
-  const long vectors = 2L * cv.batch * cv.kv_heads * max_len;
+                                 int max_len, int kinds, cudaStream_t stream) {
+  const long vectors = (long)kinds * cv.batch * cv.kv_heads * max_len;
   if (vectors <= kLatencyVectors)
-    return launch_convert_layout<D, T, D / 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
-  return launch_convert_layout<D, T, 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+    return launch_convert_layout<D, T, D / 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds,
+                                               stream);
+  return launch_convert_layout<D, T, 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds, stream);
 }
 
 template <int D>
 cudaError_t launch_convert_dim(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                                int dtype, long sb, long sh, long st, const int32_t* lengths,
-                               int max_len, cudaStream_t stream) {
+                               int max_len, int kinds, cudaStream_t stream) {
   switch (dtype) {
-    case kF32: return launch_convert_typed<D, float>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+    case kF32:
+      return launch_convert_typed<D, float>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds, stream);
     case kBF16:
-      return launch_convert_typed<D, __nv_bfloat16>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
-    case kF16: return launch_convert_typed<D, __half>(tb, cv, k, v, sb, sh, st, lengths, max_len, stream);
+      return launch_convert_typed<D, __nv_bfloat16>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds,
+                                                    stream);
+    case kF16:
+      return launch_convert_typed<D, __half>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -479,22 +486,43 @@ cudaError_t launch_quantize_append(const Tables& tb, const CacheView& cv, const 
   return cudaErrorNotSupported;
 }
 
+// Shared by the cache conversion (kinds = 2) and the weight encoding (kinds = 1).
+cudaError_t launch_convert(const Tables& tb, const CacheView& cv, const void* k, const void* v,
+                           int dtype, long stride_b, long stride_h, long stride_t,
+                           const int32_t* lengths, int max_len, int kinds, cudaStream_t stream) {
+  switch (tb.d) {
+    case 64:
+      return launch_convert_dim<64>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                    max_len, kinds, stream);
+    case 128:
+      return launch_convert_dim<128>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                     max_len, kinds, stream);
+    case 256:
+      return launch_convert_dim<256>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
+                                     max_len, kinds, stream);
+  }
+  return cudaErrorNotSupported;
+}
+
 cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const void* k,
                                   const void* v, int dtype, long stride_b, long stride_h,
                                   long stride_t, const int32_t* lengths, int max_len,
                                   cudaStream_t stream) {
-  switch (tb.d) {
-    case 64:
-      return launch_convert_dim<64>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
-                                    max_len, stream);
-    case 128:
-      return launch_convert_dim<128>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
-                                     max_len, stream);
-    case 256:
-      return launch_convert_dim<256>(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths,
-                                     max_len, stream);
-  }
-  return cudaErrorNotSupported;
+  return launch_convert(tb, cv, k, v, dtype, stride_b, stride_h, stride_t, lengths, max_len, 2,
+                        stream);
+}
+
+cudaError_t launch_weights_quantize(const Tables& tb, const void* w, int dtype, int rows, int k,
+                                    uint8_t* codes, uint16_t* norms, cudaStream_t stream) {
+  Tables t = tb;
+  t.qjl = 0;  // weights carry only the MSE codes
+  CacheView cv = {};
+  cv.k_codes = codes;  // block j of row n is "token" n of "head" j
+  cv.k_norm = norms;
+  cv.batch = 1;
+  cv.kv_heads = k / tb.d;
+  cv.capacity = rows;
+  return launch_convert(t, cv, w, w, dtype, 0, tb.d, k, nullptr, rows, 1, stream);
 }
 
 }  // namespace tq

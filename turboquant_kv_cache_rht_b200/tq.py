@@ -28,6 +28,7 @@ TQ_FLAG_CAPACITY = 1
 TQ_FLAG_MAXCTX = 2
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append", "tq_quantize_cache",
+           "tq_weights_quantize", "tq_lut_matmul_workspace_bytes", "tq_lut_matmul",
            "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_noalloc",
            "tq_free", "tq_last_error")
 
@@ -62,6 +63,14 @@ lib.tq_quantize_append.restype = C.c_int
 lib.tq_quantize_cache.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_void_p, C.c_int,
                                   C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_int, C.c_void_p]
 lib.tq_quantize_cache.restype = C.c_int
+lib.tq_weights_quantize.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
+                                    C.c_void_p, C.c_void_p]
+lib.tq_weights_quantize.restype = C.c_int
+lib.tq_lut_matmul_workspace_bytes.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int]
+lib.tq_lut_matmul_workspace_bytes.restype = C.c_size_t
+lib.tq_lut_matmul.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                              C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+lib.tq_lut_matmul.restype = C.c_int
 lib.tq_decode_workspace_bytes.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int]
 lib.tq_decode_workspace_bytes.restype = C.c_size_t
 lib.tq_decode_attention.argtypes = [C.c_void_p, C.POINTER(tq_cache), C.c_void_p, C.c_int, C.c_int,
@@ -222,6 +231,40 @@ def tq_quantize_cache(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Tens
                                  k.stride(0), k.stride(1), k.stride(2), lengths.data_ptr(), T,
                                  _stream_ptr(stream)),
            "tq_quantize_cache")
+
+
+def tq_lut_matmul_workspace_bytes(cb: Codebook, rows: int, k: int, m: int) -> int:
+    return int(lib.tq_lut_matmul_workspace_bytes(cb.handle, rows, k, m))
+
+
+class QuantizedWeights:
+    """A weight matrix [rows, k] encoded block by block (blocks of head_dim input
+    channels, the key codec): codes [k/d, rows, k_bits*d/8], fp16 norms [k/d, rows]."""
+
+    def __init__(self, cb: Codebook, w: torch.Tensor, stream=None):
+        if w.dim() != 2 or not w.is_contiguous():
+            raise ValueError("w must be a contiguous [rows, k] CUDA tensor")
+        self.cb, (self.rows, self.k) = cb, w.shape
+        nb = self.k // cb.head_dim
+        self.codes = torch.empty(nb, self.rows, cb.layout.k_code_bytes, dtype=torch.uint8, device=w.device)
+        self.norms = torch.empty(nb, self.rows, dtype=torch.float16, device=w.device)
+        _check(lib.tq_weights_quantize(cb.handle, w.data_ptr(), _dtype_code(w), self.rows, self.k,
+                                       self.codes.data_ptr(), self.norms.data_ptr(), _stream_ptr(stream)),
+               "tq_weights_quantize")
+
+    def matmul(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """x [m, k] CUDA tensor -> float32 [m, rows] = x W_hat^T."""
+        if x.dim() != 2 or x.shape[1] != self.k or not x.is_contiguous():
+            raise ValueError(f"x must be a contiguous [m, {self.k}] tensor")
+        m = x.shape[0]
+        y = torch.empty(m, self.rows, dtype=torch.float32, device=x.device)
+        nbytes = tq_lut_matmul_workspace_bytes(self.cb, self.rows, self.k, m)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+        _check(lib.tq_lut_matmul(self.cb.handle, self.codes.data_ptr(), self.norms.data_ptr(), self.rows,
+                                 self.k, x.data_ptr(), _dtype_code(x), m, y.data_ptr(), ws.data_ptr(),
+                                 nbytes, _stream_ptr(stream)),
+               "tq_lut_matmul")
+        return y
 
 
 def tq_decode_workspace_bytes(cb: Codebook, batch: int, q_heads: int, kv_heads: int,
