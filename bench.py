@@ -51,13 +51,13 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum of both kernels).  Each entry
 # carries the digest of the decode sources it was taken with; once the kernel
 # sources change the figure no longer describes them and is reported as null.
-DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d128.cu", "tq_decode_d256.cu",
-                  "tq_internal.cuh")
+DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d64.cu", "tq_decode_d128.cu",
+                  "tq_decode_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31748096, "41795a16fa794c1b"),
-    "qjl": (566693888, "41795a16fa794c1b"),
-    "long": (353863168, "41795a16fa794c1b"),
-    "serving": (1102753280, "41795a16fa794c1b"),
+    "gqa": (31748096, "37d53387cac414f4"),
+    "qjl": (566693888, "37d53387cac414f4"),
+    "long": (353863168, "37d53387cac414f4"),
+    "serving": (1102753280, "37d53387cac414f4"),
 }
 
 
