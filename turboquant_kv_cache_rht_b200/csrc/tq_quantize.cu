@@ -272,6 +272,11 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int h = valid ? (int)(r / n_new) : 0, j = valid ? (int)(r % n_new) : 0;
 
   pdl_wait();
+  // A small append (this layout) is a grid that is resident at once: let the
+  // next kernel launch now, so that its set-up overlaps this one (it still waits
+  // for this grid's completion before reading anything).  A bulk append keeps
+  // the trigger at its end, so that waiting CTAs do not take its blocks' slots.
+  if constexpr (E < 32) pdl_trigger();
   const int base = cv.seq_lens[b];
   const bool fits = base >= 0 && base <= cv.capacity - n_new;
   if (!fits && tid == 0 && blockIdx.x == 0) atomicOr(cv.status, (int)kFlagCapacity);
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(kAppendThreads)
       cv.append_sync[b] = 0;
     }
   }
-  pdl_trigger();
+  if constexpr (E == 32) pdl_trigger();
 }
 
 // Conversion of a dense cache.  Grid: (kinds * blocks_per_kind, batch) as for
