@@ -54,10 +54,10 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d64.cu", "tq_decode_d128.cu",
                   "tq_decode_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31748096, "37d53387cac414f4"),
-    "qjl": (566693888, "37d53387cac414f4"),
-    "long": (353863168, "37d53387cac414f4"),
-    "serving": (1102753280, "37d53387cac414f4"),
+    "gqa": (31748608, "083f9a3f8c6c62ea"),
+    "qjl": (566742528, "083f9a3f8c6c62ea"),
+    "long": (353532160, "083f9a3f8c6c62ea"),
+    "serving": (1102903552, "083f9a3f8c6c62ea"),
 }
 
 

@@ -44,6 +44,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 namespace tq {
 
 constexpr int kDecWarps = 4;
@@ -867,26 +869,45 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   }
 }
 
-// Sets the kernel's shared-memory attribute (once per device) and reports how
-// many of its CTAs fit on one SM.
-template <int D, int G, int KB, int VB, bool QJL>
-cudaError_t configure_shape(int* ctas_per_sm) {
-  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
-  auto kern = decode_kernel<D, G, KB, VB, QJL>;
-  static int configured_device = -1;
-  static int occupancy = 0;
+// Per-kernel record of the devices it has been configured on (each kernel
+// owns one: kernels of one signature share a function-pointer type, so the
+// record cannot be keyed on the type).
+struct KernelConfig {
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu;
+  int occupancy[kMaxDevices] = {};  // 0: not yet configured on that device
+};
+
+// Sets the kernel's shared-memory attribute and measures how many of its CTAs
+// fit on one SM, once per device; thread-safe (host threads may drive
+// different GPUs at once).
+template <typename Kernel>
+cudaError_t configure_kernel(KernelConfig& cfg, Kernel kern, int smem_bytes, int threads,
+                             int* ctas_per_sm) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::total);
+  if (dev < 0 || dev >= KernelConfig::kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(cfg.mu);
+  if (cfg.occupancy[dev] == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occupancy, kern, kDecThreads, Geo::total);
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem_bytes);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
+    cfg.occupancy[dev] = n > 0 ? n : 1;
   }
-  if (ctas_per_sm) *ctas_per_sm = occupancy;
+  if (ctas_per_sm) *ctas_per_sm = cfg.occupancy[dev];
   return cudaSuccess;
+}
+
+// The decode kernel of one compile-time shape: configured, and its CTAs per SM.
+template <int D, int G, int KB, int VB, bool QJL>
+cudaError_t configure_shape(int* ctas_per_sm) {
+  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
+  static KernelConfig cfg;  // one per shape
+  return configure_kernel(cfg, decode_kernel<D, G, KB, VB, QJL>, Geo::total, kDecThreads,
+                          ctas_per_sm);
 }
 
 // Launches decode_kernel for one compile-time shape (grid: plan.ctas CTAs).

@@ -292,20 +292,14 @@ cudaError_t launch_mm_shape(const Tables& tb, const uint8_t* codes, const uint16
                             float* partials, float* y, cudaStream_t stream) {
   using Geo = MmGeom<D, KB, NT>;
   auto kern = lut_matmul_kernel<D, KB, NT>;
-  static int configured_device = -1;
-  static int ctas_per_sm = 1, sms = 148;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  int ctas_per_sm = 1, sms = 0, dev = 0;
+  static KernelConfig config;  // one per shape
+  cudaError_t e = configure_kernel(config, kern, Geo::total, kMmThreads, &ctas_per_sm);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::total);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kern, kMmThreads, Geo::total);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   // one wave at the kernel's occupancy (never more CTAs than the workspace bound)
   const MatmulPlan plan = plan_lut_matmul(rows, k, m, D, std::min<long>(kMmMaxCtas, (long)std::max(ctas_per_sm, 1) * sms));
   float* out = plan.splits > 1 ? partials : y;
