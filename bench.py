@@ -462,12 +462,7 @@ def lut_matmul_bench(dev, peak_gbs: float, rows: int = 16384, k: int = 8192, bit
     wt = torch.randn(rows, k, generator=g, device=dev).bfloat16()
     cb = tq.Codebook(head_dim, bits, bits, seed=5)
     qw = tq.QuantizedWeights(cb, wt)
-    copies = [qw]
-    for _ in range(replicas - 1):
-        c = tq.QuantizedWeights.__new__(tq.QuantizedWeights)
-        c.cb, c.rows, c.k = cb, rows, k
-        c.codes, c.norms = qw.codes.clone(), qw.norms.clone()
-        copies.append(c)
+    copies = [qw] + [qw.copy() for _ in range(replicas - 1)]
     packed = qw.codes.numel() + qw.norms.numel() * 2
 
     def timed(fn, n):

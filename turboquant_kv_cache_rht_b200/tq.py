@@ -252,6 +252,13 @@ class QuantizedWeights:
                                        self.codes.data_ptr(), self.norms.data_ptr(), _stream_ptr(stream)),
                "tq_weights_quantize")
 
+    def copy(self) -> "QuantizedWeights":
+        """A second copy of the encoded weights (new device buffers)."""
+        c = QuantizedWeights.__new__(QuantizedWeights)
+        c.cb, c.rows, c.k = self.cb, self.rows, self.k
+        c.codes, c.norms = self.codes.clone(), self.norms.clone()
+        return c
+
     def matmul(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         """x [m, k] CUDA tensor -> float32 [m, rows] = x W_hat^T."""
         if x.dim() != 2 or x.shape[1] != self.k or not x.is_contiguous():
