@@ -18,7 +18,10 @@ Sources, cited by page title and section:
 * [P3] "mlx-turboquant" README -- introduction (randomized Hadamard transform
   preserves inner products, Lloyd-Max codebook), "The 1-bit QJL residual
   (unbiased inner-product estimator)" (r = Rk - k_hat, store sign(RHT2(r)) and
-  ||r||, add sqrt(pi/(2d))*||r||*<RHT2(Rq), sign(RHT2(r))> back to the score).
+  ||r||, add sqrt(pi/(2d))*||r||*<RHT2(Rq), sign(RHT2(r))> back to the score);
+  for the affine comparison codec: "Quantize the KV cache (long-context
+  inference)" (kv_group_size 64), "How it plugs in" (affine cache, rotated keys,
+  rotated query), "Measured results" and "Memory footprint over long context".
 
 Precision.  The codec is computed in IEEE binary32 with round-to-nearest-even,
 one operation at a time (numpy float32 ufuncs never fuse a multiply into an add),
@@ -33,7 +36,10 @@ rotation uses seed XOR 0x9E3779B97F4A7C15); one rotation shared by keys, values
 and all heads; a Lloyd-Max codebook for N(0, 1) applied to z = sqrt(d) * Rx /
 ||x||; a per-vector fp16 norm; codes packed as a little-endian bit stream;
 strict "<" against the boundaries (a tie goes to the lower index); sign(0) = +1;
-the QJL residual norm kept in the orthonormal rotated frame.
+the QJL residual norm kept in the orthonormal rotated frame.  Affine codec:
+groups of 64 consecutive channels, scale = (max - min)/(2^b - 1) and bias = min
+in fp16, codes rounded half to even and clamped, keys coded in the rotated frame
+and values unrotated.
 
 Parity status: every function is pinned by the CPU tests in ``tests/`` against
 closed forms, textbook tables, brute force or an independent second route; none
@@ -490,3 +496,113 @@ def kv_bits_split(kv_bits: float) -> tuple[int, int]:
     read as keys floor(b), values ceil(b).
     """
     return int(math.floor(kv_bits + 1e-9)), int(math.ceil(kv_bits - 1e-9))
+
+
+# ---------------------------------------------------------------------------
+# Rotated affine group-64 KV codec, the comparison codec ([P3] "Quantize the KV
+# cache (long-context inference)": kv_bits with kv_group_size=64; "How it plugs
+# in": the KV cache is mlx-lm's affine quantized cache with the keys rotated,
+# and the attention rotates the query and, with qjl, adds the sketch term;
+# "Measured results": plain affine KV versus the rotated one; "Memory footprint
+# over long context": the bytes per token).  Readings: a group is 64 consecutive
+# channels of a vector; per group, scale = (max - min) / (2^b - 1) and
+# bias = min, both stored as fp16, and a channel's code is
+# round((y - bias) / scale) clamped to [0, 2^b - 1]; keys are coded in the
+# rotated frame y = R k, values in their own frame (no rotation), so the
+# attention output needs no inverse rotation; the QJL sketch codes the residual
+# r = y - y_hat of the keys exactly as for the Lloyd-Max codec.
+# ---------------------------------------------------------------------------
+AFFINE_GROUP = 64
+
+
+def affine_encode(x: np.ndarray, bits: int, s1: np.ndarray | None = None,
+                  s2: np.ndarray | None = None) -> dict:
+    """Affine group-64 coding of the rows of ``x`` (float32 [N, d]).
+
+    Steps, each rounded to float32 (``s1`` None: no rotation, the plain codec):
+      1. y = H (s1 * x) * rs, rs = fp32(1 / fp32(sqrt(d)))     (= R x, rounded)
+      2. per group of 64 channels: mn = min y, mx = max y
+      3. scale16 = fp16((mx - mn) / (2^b - 1)); bias16 = fp16(mn)
+      4. idx = rint((y - bias16) / scale16), ties to even, clamped to
+         [0, 2^b - 1]; idx = 0 where scale16 == 0 (or the quotient is NaN)
+      5. codes = little-endian bit stream of idx
+    With ``s2`` (keys with the QJL sketch):
+      6. y_hat = fp32(fp32(scale16 * idx) + bias16); r = y - y_hat
+      7. rho = sqrt(pairwise sum of r_i * r_i); rnorm16 = fp16(rho)    (= ||Rk - k_hat||)
+      8. w = H (s2 * r); sign bit_i = (w_i >= 0)
+    ``meta16`` interleaves (scale16, bias16) per group: fp16 [N, 2 d / 64].
+    """
+    x = np.asarray(x, np.float32)
+    n, d = x.shape
+    ng = d // AFFINE_GROUP
+    if s1 is not None:
+        rs = np.float32(1.0) / np.sqrt(np.float32(d))
+        y = fwht(np.where(s1 < 0, -x, x)) * rs
+    else:
+        y = x.copy()
+    yg = y.reshape(n, ng, AFFINE_GROUP)
+    mn = yg.min(axis=-1)
+    mx = yg.max(axis=-1)
+    levels = np.float32((1 << bits) - 1)
+    scale16 = ((mx - mn) / levels).astype(np.float16)
+    bias16 = mn.astype(np.float16)
+    sf = scale16.astype(np.float32)[..., None]
+    bf = bias16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.rint((yg - bf) / sf)
+    t = np.where(np.isnan(t) | (sf == 0), np.float32(0), t)
+    idx = np.clip(t, 0, levels).astype(np.int64).reshape(n, d)
+    meta = np.stack([scale16, bias16], axis=-1).reshape(n, 2 * ng)
+    out = {"idx": idx, "codes": pack_codes(idx, bits), "scale16": scale16, "bias16": bias16,
+           "meta16": meta, "y": y}
+    if s2 is not None:
+        y_hat = (sf * idx.reshape(n, ng, AFFINE_GROUP).astype(np.float32) + bf).reshape(n, d)
+        r = y - y_hat
+        rho = np.sqrt(pairwise_sum_f32(r * r))
+        w = fwht(np.where(s2 < 0, -r, r))
+        sbits = (w >= 0).astype(np.int64)
+        out.update(sign_bits=sbits, signs=pack_codes(sbits, 1), rnorm16=rho.astype(np.float16))
+    return out
+
+
+def affine_dequantize(idx: np.ndarray, scale16: np.ndarray, bias16: np.ndarray) -> np.ndarray:
+    """y_hat = scale16 * idx + bias16 per group, in float64 ([N, d])."""
+    idx = np.asarray(idx, np.float64)
+    n, d = idx.shape
+    ng = d // AFFINE_GROUP
+    s = np.asarray(scale16, np.float64).reshape(n, ng, 1)
+    b = np.asarray(bias16, np.float64).reshape(n, ng, 1)
+    return (s * idx.reshape(n, ng, AFFINE_GROUP) + b).reshape(n, d)
+
+
+def affine_decode_attention(q: np.ndarray, s1: np.ndarray | None, ek: dict, ev: dict,
+                            sm_scale: float | None = None, s2: np.ndarray | None = None
+                            ) -> np.ndarray:
+    """Attention of the G query rows ``q`` [G, d] over the affine-coded tokens of one KV head.
+
+    float64: q_rot = R q (q itself when ``s1`` is None); k_hat, v_hat by
+    ``affine_dequantize``;  s_t = scale * (<q_rot, k_hat_t> + sqrt(pi/(2d)) *
+    rho16_t * <R2 q_rot, 2 b_t - 1>) (the second term with ``s2``);
+    o = softmax(s) v_hat (values are unrotated).  T = 0 gives a zero output.
+    """
+    q = np.atleast_2d(np.asarray(q, np.float64))
+    g, d = q.shape
+    if ek["idx"].shape[0] == 0:
+        return np.zeros((g, d))
+    q_rot = rht_forward(q, s1) if s1 is not None else q
+    scores = q_rot @ affine_dequantize(ek["idx"], ek["scale16"], ek["bias16"]).T
+    if s2 is not None:
+        q_hat = rht_forward(q_rot, s2)
+        sgn = 2.0 * np.asarray(ek["sign_bits"], np.float64) - 1.0
+        scores = scores + (math.sqrt(math.pi / (2 * d))
+                           * np.asarray(ek["rnorm16"], np.float64)[None, :] * (q_hat @ sgn.T))
+    scores = default_scale(d, sm_scale) * scores
+    p = np.exp(scores - scores.max(axis=-1, keepdims=True))
+    vals = affine_dequantize(ev["idx"], ev["scale16"], ev["bias16"])
+    return (p @ vals) / p.sum(axis=-1, keepdims=True)
+
+
+def affine_vector_bytes(d: int, bits: int, qjl: bool = False) -> int:
+    """Bytes stored per coded vector: codes, fp16 (scale, bias) per group, and
+    with the sketch d/8 sign bytes plus an fp16 residual norm."""
+    return bits * d // 8 + 4 * (d // AFFINE_GROUP) + ((d // 8 + 2) if qjl else 0)
