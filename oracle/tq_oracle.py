@@ -521,7 +521,8 @@ def affine_encode(x: np.ndarray, bits: int, s1: np.ndarray | None = None,
 
     Steps, each rounded to float32 (``s1`` None: no rotation, the plain codec):
       1. y = H (s1 * x) * rs, rs = fp32(1 / fp32(sqrt(d)))     (= R x, rounded)
-      2. per group of 64 channels: mn = min y, mx = max y
+      2. per group of 64 channels: mn = min y, mx = max y, each plus +0 (the
+         extremes are values: -0 and +0 are equal, and a zero extreme is +0)
       3. scale16 = fp16((mx - mn) / (2^b - 1)); bias16 = fp16(mn)
       4. idx = rint((y - bias16) / scale16), ties to even, clamped to
          [0, 2^b - 1]; idx = 0 where scale16 == 0 (or the quotient is NaN)
@@ -541,8 +542,8 @@ def affine_encode(x: np.ndarray, bits: int, s1: np.ndarray | None = None,
     else:
         y = x.copy()
     yg = y.reshape(n, ng, AFFINE_GROUP)
-    mn = yg.min(axis=-1)
-    mx = yg.max(axis=-1)
+    mn = yg.min(axis=-1) + np.float32(0.0)       # as values: a zero extreme is +0
+    mx = yg.max(axis=-1) + np.float32(0.0)
     levels = np.float32((1 << bits) - 1)
     scale16 = ((mx - mn) / levels).astype(np.float16)
     bias16 = mn.astype(np.float16)

@@ -197,3 +197,15 @@ def test_rotation_rescues_outlier_keys():
     err_plain = q @ o.affine_dequantize(plain["idx"], plain["scale16"], plain["bias16"]).T - exact
     err_rot = o.rht_forward(q, s1) @ o.affine_dequantize(rot["idx"], rot["scale16"], rot["bias16"]).T - exact
     assert np.sqrt((err_rot ** 2).mean()) < 0.7 * np.sqrt((err_plain ** 2).mean())
+
+
+def test_zero_extremes_are_positive_zero():
+    """-0 and +0 are one value: a group whose min or max is a zero stores it as +0."""
+    x = np.zeros((3, 128), np.float32)
+    x[1] = -0.0                                                       # all -0
+    x[2, :64] = np.where(np.arange(64) % 2, -0.0, 0.0)                # mixed zeros
+    x[2, 64:] = -np.linspace(-1, 0, 64, dtype=np.float32)             # 1 .. -0: min is -0
+    for s1 in (None, o.rotation_signs(1, 128)):
+        assert not np.any(o.affine_encode(x, 3, s1)["meta16"][:2].view(np.uint16) & 0x8000)
+    assert o.affine_encode(x, 3)["meta16"][2].view(np.uint16).tolist()[:2] == [0, 0]
+    assert o.affine_encode(x, 3)["meta16"][2].view(np.uint16)[3] == 0     # bias of group 1: +0
