@@ -1,6 +1,7 @@
 """Benchmark of the TurboQuant decode step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa|qjl|long|serving|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload gqa|qjl|long|serving|tiny|affine]
                     [--impl ours|reference] [--no-dense] [--no-cpu-baseline] [--lutmm]
 
 A step is one pass of the whole hot path over one batch: tq_quantize_append of
@@ -51,13 +52,12 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum of both kernels).  Each entry
 # carries the digest of the decode sources it was taken with; once the kernel
 # sources change the figure no longer describes them and is reported as null.
-DECODE_SOURCES = ("tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d64.cu", "tq_decode_d128.cu",
-                  "tq_decode_d256.cu")
+DECODE_SOURCES = ("tq_internal.cuh", "tq_decode_impl.cuh", "tq_decode.cu", "tq_decode_d64.cu", "tq_decode_d128.cu",
+                  "tq_decode_d256.cu", "tq_decode_affine_d64.cu", "tq_decode_affine_d128.cu",
+                  "tq_decode_affine_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31748608, "083f9a3f8c6c62ea"),
-    "qjl": (566742528, "083f9a3f8c6c62ea"),
-    "long": (353532160, "083f9a3f8c6c62ea"),
-    "serving": (1102903552, "083f9a3f8c6c62ea"),
+    "gqa": (31754240, "28c20c72a0cb8e28"),
+    "affine": (38808064, "28c20c72a0cb8e28"),
 }
 
 
@@ -90,10 +90,16 @@ def peaks():
 # ---------------------------------------------------------------------------
 # byte model (algorithmic bytes; see the design notes)
 # ---------------------------------------------------------------------------
+def meta_bytes(w: wl.Workload) -> int:
+    """fp16 metadata per stored vector: the norm, or the affine codec's
+    (scale, bias) per group of 64 channels."""
+    return 4 * (w.head_dim // 64) if w.codebook == "affine" else 2
+
+
 def token_bytes(w: wl.Workload) -> int:
     """Packed bytes one decode reads per (token, KV head)."""
     d = w.head_dim
-    b = w.k_bits * d // 8 + 2 + w.v_bits * d // 8 + 2
+    b = w.k_bits * d // 8 + w.v_bits * d // 8 + 2 * meta_bytes(w)
     if w.qjl:
         b += d // 8 + 2
     return b
@@ -104,7 +110,7 @@ def step_bytes(w: wl.Workload, lengths) -> dict:
     d = w.head_dim
     cache = sum(lengths) * w.kv_heads * token_bytes(w)
     q_out = w.batch * w.q_heads * d * (esz + 4)
-    vec_out = (w.k_bits + w.v_bits) * d // 8 + 4 + ((d // 8 + 2) if w.qjl else 0)
+    vec_out = (w.k_bits + w.v_bits) * d // 8 + 2 * meta_bytes(w) + ((d // 8 + 2) if w.qjl else 0)
     append = w.batch * w.kv_heads * (2 * d * esz + vec_out)
     return {"decode": cache + q_out, "append": append, "total": cache + q_out + append}
 
@@ -207,7 +213,7 @@ class State:
         self.tq = tq
         self.w = w
         self.dev = device
-        self.cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed)
+        self.cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed, codebook=w.codebook)
         plan = replica_plan(w, steps_total, torch.cuda.get_device_properties(device).L2_cache_size)
         self.lengths = plan["lengths"]
         self.replicas = plan["replicas"]
@@ -366,7 +372,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "config": {"workload": w.name, "description": w.description, "batch": w.batch,
                    "q_heads": w.q_heads, "kv_heads": w.kv_heads, "head_dim": w.head_dim,
                    "context": st.lengths[0] if w.context else "ragged", "k_bits": w.k_bits,
-                   "v_bits": w.v_bits, "qjl": w.qjl, "parallelism": f"replicas x{world}",
+                   "v_bits": w.v_bits, "qjl": w.qjl, "codebook": w.codebook,
+                   "parallelism": f"replicas x{world}",
                    "l2": f"{st.replicas} rotating cache replicas "
                          f"({st.replicas * sum(st.lengths) * w.kv_heads * token_bytes(w) / 1e6:.0f} MB, > 4x L2)"},
         "ctx_tokens_per_s": round(tokens_all / (ms_max * 1e-3), 1),
@@ -412,7 +419,7 @@ def bulk_quantize_mvec(st: State, dev) -> dict:
     ms = statistics.median(times)
     esz = kk.element_size()
     lay = st.cb.layout
-    byts = vecs // 2 * (2 * w.head_dim * esz + lay.k_code_bytes + lay.v_code_bytes + 4 +
+    byts = vecs // 2 * (2 * w.head_dim * esz + lay.k_code_bytes + lay.v_code_bytes + 2 * meta_bytes(w) +
                         (lay.k_sign_bytes + 2 if w.qjl else 0))
     return {"vectors": vecs, "ms": round(ms, 4), "mvec_s": round(vecs / (ms * 1e-3) / 1e6, 1),
             "gb_s": round(byts / (ms * 1e-3) / 1e9, 1)}
@@ -584,23 +591,37 @@ class OracleUnit:
         self.o, self.np, self.w = o, np, w
         self.T = wl.context_lengths(w)[0]
         d = w.head_dim
-        self.ck, self.bk = o.codebook(w.k_bits)
-        self.cv, self.bv = o.codebook(w.v_bits)
+        self.affine = w.codebook == "affine"
+        if w.codebook == "sphere":
+            self.ck, self.bk = o.sphere_codebook(w.k_bits, d)
+            self.cv, self.bv = o.sphere_codebook(w.v_bits, d)
+        elif not self.affine:
+            self.ck, self.bk = o.codebook(w.k_bits)
+            self.cv, self.bv = o.codebook(w.v_bits)
         self.s1 = o.rotation_signs(w.rht_seed, d)
         self.s2 = o.rotation_signs(w.rht_seed, d, second=True) if w.qjl else None
         k, v = wl.kv_unit(w, 0, 0, self.T)
-        self.ek = o.encode(k.float().numpy(), self.s1, self.ck, self.bk, w.k_bits, self.s2)
-        self.ev = o.encode(v.float().numpy(), self.s1, self.cv, self.bv, w.v_bits)
+        self.ek, self.ev = self._encode(k.float().numpy(), v.float().numpy())
         kn, vn = wl.kv_step(w, 0)
         self.k_new = kn[0, 0].float().numpy()
         self.v_new = vn[0, 0].float().numpy()
         self.q = wl.queries(w, 0)[0, :w.group].float().numpy().astype(np.float64)
 
+    def _encode(self, k, v):
+        o, w = self.o, self.w
+        if self.affine:
+            return o.affine_encode(k, w.k_bits, self.s1, self.s2), o.affine_encode(v, w.v_bits)
+        return (o.encode(k, self.s1, self.ck, self.bk, w.k_bits, self.s2),
+                o.encode(v, self.s1, self.cv, self.bv, w.v_bits))
+
     def step(self):
         """Append one token (encode K and V) and decode the unit's G heads."""
-        o, np, w = self.o, self.np, self.w
-        ek1 = o.encode(self.k_new, self.s1, self.ck, self.bk, w.k_bits, self.s2)
-        ev1 = o.encode(self.v_new, self.s1, self.cv, self.bv, w.v_bits)
+        o, np = self.o, self.np
+        ek1, ev1 = self._encode(self.k_new, self.v_new)
+        if self.affine:
+            cat = lambda a, b: {key: np.concatenate([a[key], b[key]]) for key in a if key in b}
+            return o.affine_decode_attention(self.q, self.s1, cat(self.ek, ek1), cat(self.ev, ev1),
+                                             s2=self.s2)
         kw = {}
         if self.s2 is not None:
             kw = dict(s2=self.s2, k_sign_bits=np.concatenate([self.ek["sign_bits"], ek1["sign_bits"]]),
@@ -614,7 +635,7 @@ class OracleUnit:
         w = self.w
         esz = {"f32": 4, "bf16": 2, "f16": 2}[w.dtype]
         d = w.head_dim
-        vec_out = (w.k_bits + w.v_bits) * d // 8 + 4 + ((d // 8 + 2) if w.qjl else 0)
+        vec_out = (w.k_bits + w.v_bits) * d // 8 + 2 * meta_bytes(w) + ((d // 8 + 2) if w.qjl else 0)
         return (self.T + 1) * token_bytes(w) + w.group * d * (esz + 4) + 2 * d * esz + vec_out
 
 

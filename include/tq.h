@@ -67,9 +67,21 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  *       fixed x, sqrt(d) (R x)_i / ||x|| is sqrt(d) times a coordinate of a
  *       uniformly random unit vector of R^d, with density proportional to
  *       (1 - z^2/d)^((d-3)/2) on |z| < sqrt(d); it depends on head_dim and
- *       tends to N(0, 1) as head_dim grows. */
+ *       tends to N(0, 1) as head_dim grows.
+ *   TQ_CODEBOOK_AFFINE : the comparison codec of the "mlx-turboquant" README
+ *       ("Quantize the KV cache (long-context inference)", kv_group_size 64;
+ *       "How it plugs in": an affine quantized cache whose keys are rotated).
+ *       Keys are coded in the rotated frame y = R k, values as they are.  Per
+ *       group of 64 consecutive channels, scale = (max - min) / (2^bits - 1)
+ *       and bias = min, both fp16; a channel's code is round((y - bias) / scale),
+ *       ties to even, clamped to [0, 2^bits - 1] (0 when scale is 0), and
+ *       y_hat = scale * code + bias.  With qjl the key sketch codes the
+ *       residual y - y_hat as for the other codebooks.  The tables hold the
+ *       integer levels 0 .. 2^bits - 1 (centroids) and their midpoints.
+ *       Inputs are expected to be finite. */
 #define TQ_CODEBOOK_GAUSSIAN 0
 #define TQ_CODEBOOK_SPHERE 1
+#define TQ_CODEBOOK_AFFINE 2
 
 /* Codec parameters.
  *   head_dim : d, 64, 128 or 256
@@ -77,8 +89,8 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  *   qjl      : 1 = keys also carry the 1-bit QJL residual sketch
  *   seed     : seeds the sign vectors of R (and of R2 = RHT2 for QJL).  One R
  *              is shared by keys, values, all heads and all batch rows.
- *   codebook : TQ_CODEBOOK_GAUSSIAN (0, the default when zero-initialized) or
- *              TQ_CODEBOOK_SPHERE. */
+ *   codebook : TQ_CODEBOOK_GAUSSIAN (0, the default when zero-initialized),
+ *              TQ_CODEBOOK_SPHERE or TQ_CODEBOOK_AFFINE. */
 typedef struct {
   int head_dim;
   int k_bits;
@@ -93,6 +105,9 @@ typedef struct {
   size_t k_code_bytes;   /* k_bits * head_dim / 8 */
   size_t v_code_bytes;   /* v_bits * head_dim / 8 */
   size_t k_sign_bytes;   /* head_dim / 8 with QJL, else 0 */
+  size_t norm_halves;    /* fp16 entries per vector in k_norm and v_norm: 1 (the
+                            norm), or 2 * head_dim / 64 for TQ_CODEBOOK_AFFINE
+                            (scale, bias of each group, in channel order) */
 } tq_layout;
 
 typedef struct tq_codebook tq_codebook;  /* opaque, host memory, owned by the library */
@@ -103,7 +118,8 @@ typedef struct tq_codebook tq_codebook;  /* opaque, host memory, owned by the li
  *   k_codes : uint8 [batch][kv_heads][capacity][k_code_bytes]
  *   v_codes : uint8 [batch][kv_heads][capacity][v_code_bytes]
  *   k_signs : uint8 [batch][kv_heads][capacity][k_sign_bytes] (QJL only, else NULL)
- *   k_norm, v_norm : fp16 bit patterns [batch][kv_heads][capacity] (||x||)
+ *   k_norm, v_norm : fp16 bit patterns [batch][kv_heads][capacity][norm_halves]
+ *                    (||x||; or the affine codec's (scale, bias) pairs)
  *   k_rnorm : fp16 bit patterns [batch][kv_heads][capacity] (QJL ||Rk - k_hat||, else NULL)
  *   seq_lens : int32 [batch], tokens currently stored per batch row
  *   status   : one int32, sticky TQ_FLAG_* bits (caller clears it)
@@ -150,6 +166,12 @@ tq_status tq_codebook_tables(const tq_codebook* cb, float* k_centroids, float* k
  *   z = u * (1/n) (0 when n == 0);  code_i = #{j : boundary_j < z_i};
  *   QJL keys: r = u - fp16(n) * c[code]; ||r||/sqrt(d) stored fp16;
  *             sign bit_i = (H (s2 * r))_i >= 0.
+ * TQ_CODEBOOK_AFFINE instead (same rounding discipline):
+ *   y = u * fp32(1 / fp32(sqrt(d))) for keys, y = x for values; per group of
+ *   64 channels (min and max as values, a zero extreme being +0)
+ *   scale = fp16((max y - min y) / (2^b - 1)), bias = fp16(min y),
+ *   code_i = rint((y_i - bias) / scale) clamped (0 when scale == 0);
+ *   QJL keys: r = y - (scale * code + bias); ||r|| stored fp16; sign bits as above.
  * A batch row whose append would pass `capacity` is skipped and sets
  * TQ_FLAG_CAPACITY.  n_new == 0 is a no-op.  NaN/Inf inputs are undefined; a
  * norm above 65504 stores an infinite fp16 norm. */
@@ -204,7 +226,9 @@ size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, 
  *   s_t = scale * (<Rq, n_t c_K[code_t]/sqrt(d)>
  *                  + sqrt(pi/(2d)) * rho_t * <R2 R q, 2 bit_t - 1>)   (QJL term if enabled)
  *   out = R^T (sum_t softmax(s)_t * m_t c_V[vcode_t] / sqrt(d)),
- * never writing a dequantized cache.  seq_lens[b] == 0 gives zeros.  The
+ * and with TQ_CODEBOOK_AFFINE, y_hat = scale * code + bias of each group:
+ *   s_t = scale * (<Rq, k_hat_t> + the same QJL term),  out = sum_t softmax(s)_t v_hat_t
+ * (values are not rotated), never writing a dequantized cache.  seq_lens[b] == 0 gives zeros.  The
  * result is deterministic (fixed-order merge of the splits). */
 tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, const void* q,
                               tq_dtype dtype, int q_heads, float softmax_scale, int max_ctx,
@@ -245,7 +269,9 @@ tq_status tq_decode_attention_noalloc(const tq_codebook* cb, const tq_cache* cac
  * tq_weights_quantize: w DEVICE [rows][k] of `dtype`, 16-byte aligned;
  *   codes DEVICE uint8 [k / head_dim][rows][k_bits * head_dim / 8];
  *   norms DEVICE fp16 bits [k / head_dim][rows]; both 16-byte aligned.
- *   rows must be a multiple of 16 and k a multiple of head_dim. */
+ *   rows must be a multiple of 16 and k a multiple of head_dim.
+ *   A TQ_CODEBOOK_AFFINE codebook is rejected (TQ_ERR_UNSUPPORTED) by this
+ *   call and by tq_lut_matmul. */
 tq_status tq_weights_quantize(const tq_codebook* cb, const void* w, tq_dtype dtype, int rows, int k,
                               uint8_t* codes, uint16_t* norms, void* stream);
 

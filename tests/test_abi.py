@@ -63,7 +63,7 @@ def test_layout_bytes():
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(head_dim=512), dict(k_bits=1),
-                                 dict(v_bits=5), dict(qjl=2), dict(codebook=2), dict(codebook=-1)])
+                                 dict(v_bits=5), dict(qjl=2), dict(codebook=3), dict(codebook=-1)])
 def test_codebook_rejects_bad_params(bad):
     p = dict(head_dim=128, k_bits=3, v_bits=4, qjl=0, seed=0, codebook=0)
     p.update(bad)
@@ -72,6 +72,28 @@ def test_codebook_rejects_bad_params(bad):
     assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_ERR_INVALID
     assert not h.value
     assert tq.tq_last_error()
+
+
+def test_affine_layout_matches_the_pages_memory_table(golden):
+    """The library's per-vector bytes for the affine codec reproduce the
+    "Memory footprint over long context" KB/token figures (the fp16 row fixes
+    the cached channels per token; head_dim 128)."""
+    rows = {r[0]: (int(r[1]), int(r[2]), int(r[3]), float(r[4])) for r in golden("kv_memory_footprint.txt")}
+    vectors = rows["fp16"][3] * 1024 / (2 * 2) / 128
+    for name in ("affine4", "turboquant4", "turboquant3_qjl"):
+        kb, vb, qjl, want = rows[name]
+        lay = tq.Codebook(128, kb, vb, qjl=bool(qjl), codebook="affine").layout
+        per_vec = (lay.k_code_bytes + lay.v_code_bytes + lay.k_sign_bytes + (2 if qjl else 0)
+                   + 2 * (2 * lay.norm_halves))                     # fp16 metadata of K and V
+        assert abs(per_vec * vectors / 1024 - want) <= 0.05, name
+    assert tq.Codebook(128, 4, 4).layout.norm_halves == 1
+    assert tq.Codebook(256, 2, 3, codebook="affine").layout.norm_halves == 8
+
+
+def test_affine_tables_are_integer_levels():
+    t = tq.Codebook(64, 3, 4, codebook="affine").tables()
+    assert t["k_centroids"].tolist() == list(range(8)) and t["v_centroids"].tolist() == list(range(16))
+    assert t["k_boundaries"].tolist() == [j + 0.5 for j in range(7)]
 
 
 def test_head_dim_64_layout():
@@ -144,6 +166,9 @@ def test_weights_validation():
     assert wq(dtype=9) == tq.TQ_ERR_INVALID
     assert wq(w=0) == tq.TQ_ERR_INVALID
     assert wq(codes=(1 << 13) + 4) == tq.TQ_ERR_INVALID
+    acb = tq.Codebook(128, 4, 4, codebook="affine")                # weights take Lloyd-Max codes
+    assert tq.lib.tq_weights_quantize(acb.handle, 1 << 12, 1, 64, 512, 1 << 13, 1 << 14,
+                                      None) == tq.TQ_ERR_UNSUPPORTED
     mm = lambda rows=64, k=512, m=1, ws=0, nbytes=0, y=1 << 15: tq.lib.tq_lut_matmul(
         cb.handle, 1 << 13, 1 << 14, rows, k, 1 << 12, 1, m, y, ws, nbytes, None)
     assert mm(m=0) == tq.TQ_ERR_INVALID

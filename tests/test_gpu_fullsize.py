@@ -27,13 +27,14 @@ CASES = {
     "long": [(0, 0), (0, 3)],
     "serving": [(0, 0), (31, 7), (17, 2)],
     "tiny": [(0, 0)],
+    "affine": [(0, 0), (0, 7), (0, 2)],
 }
 
 
 def _run_step(w, dev):
     plan = bench.replica_plan(w, bench.default_steps_total(), torch.cuda.get_device_properties(dev).L2_cache_size)
     lengths, cap, max_ctx = plan["lengths"], plan["capacity"], plan["max_ctx"]
-    cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed)
+    cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed, codebook=w.codebook)
     cache = tq.Cache(cb, w.batch, w.kv_heads, cap, dev)
     tmax = max(lengths)
     for h in range(w.kv_heads):          # bulk prefill, one KV head at a time (as bench.py)
@@ -66,7 +67,7 @@ def test_full_size_sampled_units(name):
     w = wl.WORKLOADS[name]
     dev = torch.device("cuda", 0)
     cache, out, lengths, k_new, v_new, q = _run_step(w, dev)
-    tb = oracle_tables(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed)
+    tb = oracle_tables(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed, codebook=w.codebook)
     G = w.group
     for b, h in CASES[name]:
         k, v = wl.kv_unit(w, b, h, lengths[b])

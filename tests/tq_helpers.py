@@ -12,6 +12,10 @@ DEC_TOL = 2e-3   # decode: per row, max |gpu - oracle| <= DEC_TOL * max |oracle|
 
 
 def oracle_tables(head_dim, k_bits, v_bits, qjl, seed, codebook="gaussian"):
+    if codebook == "affine":      # the affine group-64 comparison codec: signs only
+        s2 = o.rotation_signs(seed, head_dim, second=True) if qjl else None
+        return dict(affine=True, s1=o.rotation_signs(seed, head_dim), s2=s2, k_bits=k_bits,
+                    v_bits=v_bits)
     book = (lambda b: o.codebook(b)) if codebook == "gaussian" else (lambda b: o.sphere_codebook(b, head_dim))
     ck, bk = book(k_bits)
     cv, bv = book(v_bits)
@@ -24,12 +28,18 @@ def oracle_encode_unit(tb, k, v):
     """Oracle encoding of one (batch row, KV head): k, v torch [T, d] (any float dtype)."""
     kf = k.float().numpy()
     vf = v.float().numpy()
+    if tb.get("affine"):          # keys rotated, values as they are
+        return (o.affine_encode(kf, tb["k_bits"], tb["s1"], tb["s2"]),
+                o.affine_encode(vf, tb["v_bits"]))
     ek = o.encode(kf, tb["s1"], tb["ck"], tb["bk"], tb["k_bits"], tb["s2"])
     ev = o.encode(vf, tb["s1"], tb["cv"], tb["bv"], tb["v_bits"])
     return ek, ev
 
 
 def oracle_decode_unit(tb, q_rows, ek, ev, scale=None):
+    if tb.get("affine"):
+        return o.affine_decode_attention(q_rows.float().numpy().astype(np.float64), tb["s1"], ek, ev,
+                                         sm_scale=scale, s2=tb["s2"])
     kw = {}
     if tb["s2"] is not None:
         kw = dict(s2=tb["s2"], k_sign_bits=ek["sign_bits"], k_rnorm16=ek["rnorm16"])

@@ -188,6 +188,16 @@ bool build_codebook(int bits, int kind, int d, float* cent, float* bnd) {
   return true;
 }
 
+// Affine codec tables: the integer levels 0 .. 2^bits - 1 and their midpoints
+// (the decode kernel's pair tables turn code pairs into these levels).
+void build_affine_levels(int bits, float* cent, float* bnd) {
+  const int levels = 1 << bits;
+  for (int j = 0; j < 16; ++j) {
+    cent[j] = j < levels ? (float)j : 0.0f;
+    bnd[j] = j + 1 < levels ? (float)j + 0.5f : INFINITY;
+  }
+}
+
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the sign of channel i is the
 // top bit of the i-th output.
 void build_signs(uint64_t state, int d, uint32_t* mask) {
@@ -210,8 +220,10 @@ tq_status check_params(const tq_params* p) {
     return fail(TQ_ERR_INVALID, "k_bits=%d v_bits=%d: each must be 2, 3 or 4", p->k_bits,
                 p->v_bits);
   if (p->qjl != 0 && p->qjl != 1) return fail(TQ_ERR_INVALID, "qjl must be 0 or 1");
-  if (p->codebook != TQ_CODEBOOK_GAUSSIAN && p->codebook != TQ_CODEBOOK_SPHERE)
-    return fail(TQ_ERR_INVALID, "codebook %d: must be TQ_CODEBOOK_GAUSSIAN or TQ_CODEBOOK_SPHERE",
+  if (p->codebook != TQ_CODEBOOK_GAUSSIAN && p->codebook != TQ_CODEBOOK_SPHERE &&
+      p->codebook != TQ_CODEBOOK_AFFINE)
+    return fail(TQ_ERR_INVALID,
+                "codebook %d: must be TQ_CODEBOOK_GAUSSIAN, TQ_CODEBOOK_SPHERE or TQ_CODEBOOK_AFFINE",
                 p->codebook);
   return TQ_OK;
 }
@@ -294,8 +306,12 @@ tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout
   t.v_bits = params->v_bits;
   t.qjl = params->qjl;
   const int kind = params->codebook, d = params->head_dim;
-  if (!build_codebook(params->k_bits, kind, d, t.k_cent, t.k_bnd) ||
-      !build_codebook(params->v_bits, kind, d, t.v_cent, t.v_bnd)) {
+  t.affine = kind == TQ_CODEBOOK_AFFINE;
+  if (t.affine) {
+    build_affine_levels(params->k_bits, t.k_cent, t.k_bnd);
+    build_affine_levels(params->v_bits, t.v_cent, t.v_bnd);
+  } else if (!build_codebook(params->k_bits, kind, d, t.k_cent, t.k_bnd) ||
+             !build_codebook(params->v_bits, kind, d, t.v_cent, t.v_bnd)) {
     delete cb;
     return fail(TQ_ERR_INVALID, "Lloyd-Max iteration did not converge");
   }
@@ -305,6 +321,7 @@ tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout
     layout->k_code_bytes = (size_t)params->k_bits * params->head_dim / 8;
     layout->v_code_bytes = (size_t)params->v_bits * params->head_dim / 8;
     layout->k_sign_bytes = params->qjl ? (size_t)params->head_dim / 8 : 0;
+    layout->norm_halves = t.affine ? (size_t)2 * params->head_dim / tq::kAffineGroup : 1;
   }
   *out = cb;
   return ok();
@@ -374,6 +391,8 @@ tq_status tq_quantize_cache(const tq_codebook* cb, const tq_cache* cache, const 
 
 static tq_status check_weights(const tq_codebook* cb, int rows, int k, tq_dtype dtype) {
   if (!cb) return fail(TQ_ERR_INVALID, "codebook is NULL");
+  if (cb->tables.affine)
+    return fail(TQ_ERR_UNSUPPORTED, "the weights regime takes a Lloyd-Max codebook, not the affine codec");
   if (rows <= 0 || rows % 16) return fail(TQ_ERR_INVALID, "rows %d: a positive multiple of 16", rows);
   const int d = cb->params.head_dim;
   if (k <= 0 || k % d) return fail(TQ_ERR_INVALID, "k %d: a positive multiple of head_dim %d", k, d);

@@ -164,6 +164,49 @@ __device__ __forceinline__ int bucket(float z, const float (&p)[8]) {
   return pos ? H + c : H - 1 - c;
 }
 
+// Stores the lane's LB = B * E code bits (words[], code e at bit B * e) into
+// the packed row at stream bit g * LB.
+template <int D, int E, int B>
+__device__ __forceinline__ void store_codes(const uint32_t (&words)[(B * E + 31) / 32], int g,
+                                            int lane, bool store, uint8_t* codes_row,
+                                            uint32_t* pack) {
+  constexpr int LB = B * E;
+  if constexpr (LB % 32 == 0) {
+    if (store) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(codes_row + g * (LB / 8));
+#pragma unroll
+      for (int w = 0; w < LB / 32; ++w) dst[w] = words[w];
+    }
+  } else {
+    pack_store_shared(pack, B * D / 32, words[0], LB, lane, store,
+                      reinterpret_cast<uint32_t*>(codes_row));
+  }
+}
+
+// QJL sketch of the key residual r held in u: rnorm = fp16(||r|| / rdiv) and
+// the sign bits of H (s2 * r) (bit set: >= 0).
+template <int D, int E>
+__device__ __forceinline__ void store_sketch(float (&u)[E], const Tables& tb, float rdiv, int g,
+                                             int lane, bool store, uint8_t* signs_row,
+                                             uint16_t* rnorm, uint32_t* pack) {
+  constexpr int GL = D / E;
+  float sq[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) sq[e] = __fmul_rn(u[e], u[e]);
+  const float rho = __fdiv_rn(__fsqrt_rn(tree_sum<E, GL>(sq)), rdiv);
+  flip_signs<E>(u, tb.s2, g);
+  fwht<E, GL>(u, lane);
+  uint32_t sbits = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) sbits |= (u[e] >= 0.f ? 1u : 0u) << e;
+  if constexpr (E % 32 == 0) {
+    if (store) reinterpret_cast<uint32_t*>(signs_row)[g] = sbits;
+  } else {
+    pack_store_shared(pack, D / 32, sbits, E, lane, store, reinterpret_cast<uint32_t*>(signs_row));
+  }
+  if (store && g == 0) *rnorm = __half_as_ushort(__float2half_rn(rho));
+}
+
 // Encodes the vector whose E-channel slice this lane holds in u (fp32) and
 // stores codes, norm and, for QJL keys, the sketch.  g is the lane's index in
 // its group of D / E lanes; `store` is false for lanes of a group past the
@@ -210,35 +253,76 @@ __device__ __forceinline__ void encode_store(float (&u)[E], const Tables& tb, bo
     // QJL keys: the residual r = u - fp16(n) * c[code] replaces u
     if (qjl) u[e] = __fsub_rn(u[e], __fmul_rn(n16f, s_kcent[c]));
   }
-  if constexpr (LB % 32 == 0) {
-    if (store) {
-      uint32_t* dst = reinterpret_cast<uint32_t*>(codes_row + g * (LB / 8));
-#pragma unroll
-      for (int w = 0; w < LB / 32; ++w) dst[w] = words[w];
-    }
-  } else {
-    pack_store_shared(pack, B * D / 32, words[0], LB, lane, store,
-                      reinterpret_cast<uint32_t*>(codes_row));
-  }
+  store_codes<D, E, B>(words, g, lane, store, codes_row, pack);
   if (store && g == 0) *norm = __half_as_ushort(n16);
 
   // 6.-8. QJL sketch of keys: rho = ||r|| / sqrt(d); sign bits of H (s2 * r)
-  if (qjl) {
-#pragma unroll
-    for (int e = 0; e < E; ++e) sq[e] = __fmul_rn(u[e], u[e]);
-    const float rho = __fdiv_rn(__fsqrt_rn(tree_sum<E, GL>(sq)), __fsqrt_rn((float)D));
-    flip_signs<E>(u, tb.s2, g);
+  if (qjl) store_sketch<D, E>(u, tb, __fsqrt_rn((float)D), g, lane, store, signs_row, rnorm, pack);
+}
+
+// The affine group-64 comparison codec ("mlx-turboquant" README, "Quantize
+// the KV cache (long-context inference)" and "How it plugs in": an affine
+// quantized cache with group size 64 whose keys are rotated).  Keys are coded
+// in the rotated frame y = u * fp32(1/sqrt(d)), values as they are.  Per group
+// of 64 channels (64 / E adjacent lanes): scale = fp16((max - min) / (2^B - 1)),
+// bias = fp16(min), code = rint((y - bias) / scale) clamped to [0, 2^B - 1]
+// (0 when scale is 0; fminf/fmaxf send a NaN quotient to 0).  meta receives
+// the groups' (scale, bias) pairs, one 32-bit word each.  QJL keys then sketch
+// r = y - (scale * code + bias) like the Lloyd-Max codec (||r||, undivided).
+template <int D, int E, int B>
+__device__ __forceinline__ void encode_affine_store(float (&u)[E], const Tables& tb, bool is_v,
+                                                    int g, int lane, bool store,
+                                                    uint8_t* codes_row, uint32_t* meta,
+                                                    uint8_t* signs_row, uint16_t* rnorm,
+                                                    uint32_t* pack) {
+  constexpr int GL = D / E;
+  constexpr int LB = B * E;
+  constexpr int GG = kAffineGroup / E;  // lanes per channel group (2 .. 32)
+  static_assert(E <= kAffineGroup && GG <= GL, "a lane's channels lie in one group");
+  constexpr float kLevels = (float)((1 << B) - 1);
+
+  if (!is_v) {
+    flip_signs<E>(u, tb.s1, g);
     fwht<E, GL>(u, lane);
-    uint32_t sbits = 0;
+    const float rs = __fdiv_rn(1.0f, __fsqrt_rn((float)D));
 #pragma unroll
-    for (int e = 0; e < E; ++e) sbits |= (u[e] >= 0.f ? 1u : 0u) << e;
-    if constexpr (E % 32 == 0) {
-      if (store) reinterpret_cast<uint32_t*>(signs_row)[g] = sbits;
-    } else {
-      pack_store_shared(pack, D / 32, sbits, E, lane, store, reinterpret_cast<uint32_t*>(signs_row));
-    }
-    if (store && g == 0) *rnorm = __half_as_ushort(__float2half_rn(rho));
+    for (int e = 0; e < E; ++e) u[e] = __fmul_rn(u[e], rs);
   }
+  // group minimum and maximum (exact: no rounding, so any order)
+  float mn = u[0], mx = u[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) {
+    mn = fminf(mn, u[e]);
+    mx = fmaxf(mx, u[e]);
+  }
+#pragma unroll
+  for (int m = 1; m < GG; m <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+  }
+  // as values: -0 and +0 compare equal, so a zero extreme is taken as +0
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kLevels));
+  const __half b16 = __float2half_rn(mn);
+  const float sf = __half2float(s16), bf = __half2float(b16);
+  const bool qjl = !is_v && tb.qjl;
+  uint32_t words[(LB + 31) / 32];
+#pragma unroll
+  for (int w = 0; w < (LB + 31) / 32; ++w) words[w] = 0u;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float t = sf == 0.f ? 0.f : rintf(__fdiv_rn(__fsub_rn(u[e], bf), sf));
+    const int c = (int)fminf(fmaxf(t, 0.f), kLevels);
+    const int bit = B * e, w = bit >> 5, s = bit & 31;
+    words[w] |= (uint32_t)c << s;
+    if (s + B > 32) words[w + 1] |= (uint32_t)c >> (32 - s);
+    if (qjl) u[e] = __fsub_rn(u[e], __fadd_rn(__fmul_rn(sf, (float)c), bf));
+  }
+  store_codes<D, E, B>(words, g, lane, store, codes_row, pack);
+  if (store && g % GG == 0)
+    meta[g / GG] = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(b16) << 16);
+  if (qjl) store_sketch<D, E>(u, tb, 1.0f, g, lane, store, signs_row, rnorm, pack);
 }
 
 }  // namespace codec

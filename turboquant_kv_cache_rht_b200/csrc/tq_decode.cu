@@ -2,6 +2,7 @@
 #include "tq_decode_impl.cuh"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace tq {
 
@@ -35,8 +36,9 @@ static_assert(kMaxTargetCtas <= kMaxParts, "a unit's partials must fit the merge
 // inverse rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
 // w_s = 2^(m_s - max m) ("How to Use TurboQuant ...", "What is TurboQuant?":
 // _rht_inverse; the 1/d collects the rotation's and the dequantization's
-// 1/sqrt(d)).  The partials are those of the CTAs whose tile ranges meet the
-// unit's (the partition of DecodePlan, recomputed here from the lengths).
+// 1/sqrt(d)).  The affine codec's values are not rotated: o = sum / l.  The
+// partials are those of the CTAs whose tile ranges meet the unit's (the
+// partition of DecodePlan, recomputed here from the lengths).
 // Every partial is loaded at once (warp w takes partials w, w+8, ..., lane l
 // channels l*d/32 ..), so the merge costs one memory round trip; all
 // reductions run in a fixed order.
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (int e = 0; e < E; ++e) part[warp][lane * E + e] = a[e];
   __syncthreads();
   if (warp == 0) {
-    const float inv = 1.0f / (l * (float)D);
+    const float inv = 1.0f / (tb.affine ? l : l * (float)D);
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -182,12 +184,17 @@ __global__ void __launch_bounds__(kCombineThreads)
       for (int w = 1; w < W; ++w) v += part[w][ch];
       u[e] = v;
     }
-    warp_fwht<E>(u, lane);
+    if (tb.affine) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int ch = lane * E + e;
-      const float v = u[e] * inv;
-      dst[ch] = ((tb.s1[ch >> 5] >> (ch & 31)) & 1u) ? -v : v;
+      for (int e = 0; e < E; ++e) dst[lane * E + e] = u[e] * inv;
+    } else {
+      warp_fwht<E>(u, lane);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int ch = lane * E + e;
+        const float v = u[e] * inv;
+        dst[ch] = ((tb.s1[ch >> 5] >> (ch & 31)) & 1u) ? -v : v;
+      }
     }
   }
   pdl_trigger();
@@ -227,18 +234,32 @@ cudaError_t launch_decode(const Tables& tb, const CacheView& cv, const void* q, 
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = tb.d == 64    ? decode_occupancy_dim<64>(tb, group, &ctas_per_sm)
-      : tb.d == 128 ? decode_occupancy_dim<128>(tb, group, &ctas_per_sm)
-                    : decode_occupancy_dim<256>(tb, group, &ctas_per_sm);
+  if (tb.affine)
+    e = tb.d == 64    ? decode_occupancy_dim<64, true>(tb, group, &ctas_per_sm)
+        : tb.d == 128 ? decode_occupancy_dim<128, true>(tb, group, &ctas_per_sm)
+                      : decode_occupancy_dim<256, true>(tb, group, &ctas_per_sm);
+  else
+    e = tb.d == 64    ? decode_occupancy_dim<64, false>(tb, group, &ctas_per_sm)
+        : tb.d == 128 ? decode_occupancy_dim<128, false>(tb, group, &ctas_per_sm)
+                      : decode_occupancy_dim<256, false>(tb, group, &ctas_per_sm);
   if (e != cudaSuccess) return e;
   const long target = std::min<long>(kMaxTargetCtas, (long)std::max(ctas_per_sm, 1) * sms);
   const DecodePlan plan = plan_decode(cv.batch, cv.kv_heads, max_ctx, target);
+  auto launch = [&](auto dim, auto aff) {
+    return launch_decode_dim<decltype(dim)::value, decltype(aff)::value>(
+        tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+  };
+  using T = std::true_type;
+  using F = std::false_type;
+  using D64 = std::integral_constant<int, 64>;
+  using D128 = std::integral_constant<int, 128>;
+  using D256 = std::integral_constant<int, 256>;
   if (tb.d == 64)
-    e = launch_decode_dim<64>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+    e = tb.affine ? launch(D64{}, T{}) : launch(D64{}, F{});
   else if (tb.d == 128)
-    e = launch_decode_dim<128>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+    e = tb.affine ? launch(D128{}, T{}) : launch(D128{}, F{});
   else if (tb.d == 256)
-    e = launch_decode_dim<256>(tb, cv, q, dtype, q_heads, scale_log2, max_ctx, plan, workspace, stream);
+    e = tb.affine ? launch(D256{}, T{}) : launch(D256{}, F{});
   else
     e = cudaErrorNotSupported;
   if (e != cudaSuccess) return e;

@@ -132,6 +132,13 @@ __device__ __forceinline__ uint32_t field_scaled(const uint32_t* w, int n, int o
   return (w[wi] >> s) & mask;
 }
 
+// s * c + b on a half2 of two tokens' values (one fp16 rounding, as fma).
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t s, uint32_t c, uint32_t b) {
+  const __half2 r = __hfma2(*reinterpret_cast<const __half2*>(&s), *reinterpret_cast<const __half2*>(&c),
+                            *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // +-1.0 half2 from the two sign bits at positions 15 and 31 (bit 1 -> +1)
 __device__ __forceinline__ uint32_t sign_pair(uint32_t x) { return (x & 0x80008000u) ^ 0xBC00BC00u; }
 
@@ -166,7 +173,7 @@ constexpr int v_stride_words(int d, int bits) {
                  : d == 128 ? (bits == 4 ? 20 : 12) : (bits == 2 ? 20 : bits == 3 ? 28 : 36);
 }
 
-template <int D, int G, int KB, int VB, bool QJL>
+template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 struct DecodeGeom {
   static constexpr int NT = G > 4 ? 2 : 1;    // n-tiles of 8 columns (4 heads x {hi, lo})
   static constexpr int KBLK = D / 16;         // 16-channel k-blocks of the score MMA
@@ -194,13 +201,20 @@ struct DecodeGeom {
   static constexpr int RVL = VB <= 3 ? 5 : 4;  // log2 value copies (32 or 16)
   static constexpr int KSH = 3 + RKL;          // byte shift of a key entry index (8-byte entries)
   static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
+  // affine codec: NG groups of 64 channels, one (scale, bias) word per group
+  // and token; thread quarter qd reads channels [64 gg + 16 qd, + 16) of group gg
+  static constexpr int NG = D / kAffineGroup;
+  static constexpr int MB = AFF ? 4 * NG : 2;  // metadata bytes per token (keys or values)
+  static constexpr int QBA = 16 * KB;          // key bits per thread quarter and group
+  static constexpr int KWA = (QBA + 31) / 32;
+  static constexpr int KNWA = (QBA % 32 == 0) ? QBA / 32 : (QBA + 16 + 31) / 32;
   // one pipeline stage (bytes)
   static constexpr int offK = 0;
   static constexpr int offV = offK + kDecTile * KS * 4;
   static constexpr int offS = offV + kDecTile * VS * 4 + 16;
   static constexpr int offKN = offS + (QJL ? kDecTile * SS * 4 : 0);
-  static constexpr int offVN = offKN + kDecTile * 2;
-  static constexpr int offRN = offVN + kDecTile * 2;
+  static constexpr int offVN = offKN + kDecTile * MB;
+  static constexpr int offRN = offVN + kDecTile * MB;
   static constexpr int stage = offRN + (QJL ? kDecTile * 2 : 0);
   static constexpr int stageA = (stage + 127) / 128 * 128;
   // epilogue merge buffer, reusing the stage area: per warp m[G], l[G], O[G][D]
@@ -212,7 +226,8 @@ struct DecodeGeom {
   static constexpr int offLV = offLK + (LK << RKL) * 8;
   static constexpr int offQ = offLV + (LV << RVL) * 4;         // float [G][D] rotated query
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
-  static constexpr int offRed = offQ2 + (QJL ? G * D * 4 : 0); // float scratch
+  static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
+  static constexpr int offRed = offUs + (AFF ? (G * NG * 4 + 15) / 16 * 16 : 0);  // float scratch
   static constexpr int redFloats = (16 > 5 * G ? 16 : 5 * G) + 16;
   // work schedule: scan scratch (one 64-bit word per warp), then one chunk of
   // rows (index, 64-bit tile prefix)
@@ -337,12 +352,12 @@ __device__ __forceinline__ long long block_exclusive_scan(long long x, long long
 template <int D, int G, bool QJL>
 constexpr int decode_min_ctas() { return D <= 128 ? ((G > 4 || QJL) ? 3 : 4) : 2; }
 
-template <int D, int G, int KB, int VB, bool QJL>
+template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     decode_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                   const void* __restrict__ q, int q_dtype, int q_heads, float scale_log2,
                   int max_ctx, int nslots, float* __restrict__ ws) {
-  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
+  using Geo = DecodeGeom<D, G, KB, VB, QJL, AFF>;
   constexpr int NT = Geo::NT;
   extern __shared__ __align__(128) uint8_t smem[];
 
@@ -454,15 +469,29 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       for (int i = 0; i < NS; ++i)
         if (s_row[i] < rows) cp_async16(st + s_dst[i], sb + (s_dst[i] - Geo::offS));
     }
-    // norms: rows * 2 bytes each = rows / 8 chunks per array
-    const int c = tid & 7, arr = tid >> 3;
-    if (c < rows / 8) {
-      if (arr == 0)
-        cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
-      else if (arr == 1)
-        cp_async16(st + Geo::offVN + c * 16, reinterpret_cast<const uint8_t*>(cv.v_norm + row_slot + start) + c * 16);
-      else if (QJL && arr == 2)
-        cp_async16(st + Geo::offRN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + c * 16);
+    if constexpr (AFF) {
+      // (scale, bias) words: rows * NG per array, rows * NG / 4 chunks of 16 bytes
+      const int nc = rows * Geo::NG / 4;
+      const long mo = (row_slot + start) * (long)Geo::MB;
+      for (int c = tid; c < 2 * nc; c += kDecThreads) {
+        const bool vv = c >= nc;
+        const int cc = vv ? c - nc : c;
+        cp_async16(st + (vv ? Geo::offVN : Geo::offKN) + cc * 16,
+                   reinterpret_cast<const uint8_t*>(vv ? cv.v_norm : cv.k_norm) + mo + cc * 16);
+      }
+      if (QJL && tid < rows / 8)
+        cp_async16(st + Geo::offRN + tid * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + tid * 16);
+    } else {
+      // norms: rows * 2 bytes each = rows / 8 chunks per array
+      const int c = tid & 7, arr = tid >> 3;
+      if (c < rows / 8) {
+        if (arr == 0)
+          cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
+        else if (arr == 1)
+          cp_async16(st + Geo::offVN + c * 16, reinterpret_cast<const uint8_t*>(cv.v_norm + row_slot + start) + c * 16);
+        else if (QJL && arr == 2)
+          cp_async16(st + Geo::offRN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + c * 16);
+      }
     }
   };
 
@@ -494,6 +523,17 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     for (int e = 0; e < E; ++e) {
       qs[h * D + lane * E + e] = u[e];
       amax = fmaxf(amax, fabsf(u[e]));
+    }
+    if constexpr (AFF) {
+      // sum of the rotated query over each 64-channel group (GG lanes each)
+      constexpr int GG = kAffineGroup / E;
+      float t = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) t += u[e];
+#pragma unroll
+      for (int m = 1; m < GG; m <<= 1) t += __shfl_xor_sync(0xffffffffu, t, m);
+      if ((lane & (GG - 1)) == 0)
+        reinterpret_cast<float*>(smem + Geo::offUs)[h * Geo::NG + lane / GG] = t;
     }
     if constexpr (QJL) {
 #pragma unroll
@@ -530,7 +570,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   // score = post * (tensor-core sum): undoes the query scale and folds the
   // softmax scale, log2(e), the rotation's and the dequantization's 1/sqrt(d)
   // (and sqrt(pi/(2d)) of the QJL estimate)
-  const float kpost = scale_log2 / ((float)D * qsc);
+  // (affine: the keys are in the orthonormal frame, only the query's H is unnormalized)
+  const float kpost = AFF ? scale_log2 / (sqrtf((float)D) * qsc) : scale_log2 / ((float)D * qsc);
   const float qpost = scale_log2 * sqrtf(3.14159265358979f / (2.0f * D)) / ((float)D * qsc2);
 
   // ---- B fragments (query columns) in registers
@@ -543,7 +584,9 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     const float* r = qs + (live ? head : 0) * D;
 #pragma unroll
     for (int kb = 0; kb < Geo::KBLK; ++kb) {
-      const int c0 = qd * (D / 4) + 4 * kb;  // key slots 2q,2q+1 -> c0,c0+1; 2q+8,2q+9 -> c0+2,c0+3
+      // key slots 2q,2q+1 -> c0,c0+1; 2q+8,2q+9 -> c0+2,c0+3 (affine: k-block kb
+      // lies in group kb / 4, so every MMA sums channels of one group)
+      const int c0 = AFF ? kAffineGroup * (kb >> 2) + 16 * qd + 4 * (kb & 3) : qd * (D / 4) + 4 * kb;
       const float4 x = *reinterpret_cast<const float4*>(r + c0);
       uint32_t h01, l01, h23, l23;
       split_pair(x.x * qsc, x.y * qsc, h01, l01);
@@ -564,6 +607,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
         bq[j][kb][1] = live ? (part ? b_l : b_h) : 0u;
       }
     }
+  }
+
+  // affine: the query's group sums (times the query scale) for the bias term
+  float usc[NT][AFF ? Geo::NG : 1];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 4 * j + qd;
+#pragma unroll
+    for (int gg = 0; gg < (AFF ? Geo::NG : 1); ++gg)
+      usc[j][gg] = (AFF && head < G) ? reinterpret_cast<const float*>(smem + Geo::offUs)[head * Geo::NG + gg] * qsc : 0.f;
   }
 
   // ---- per-warp online softmax state and output accumulators
@@ -588,6 +641,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   // slab so that it overlaps that slab's score work (registers and the value
   // table only: the stage it came from may already be refilled)
   uint32_t pva[Geo::VCW], pvb[Geo::VCW], pvc[Geo::VCW], pvd[Geo::VCW], ppb[NT][2];
+  // affine: (scale, bias) half2 pairs of tokens (2q, 2q+1) and (2q+8, 2q+9)
+  uint32_t psab = 0u, pbab = 0u, pscd = 0u, pbcd = 0u;
 #pragma unroll
   for (int w = 0; w < Geo::VCW; ++w) pva[w] = pvb[w] = pvc[w] = pvd[w] = 0u;
 #pragma unroll
@@ -601,10 +656,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       uint32_t e0, o0, e1, o1;
       value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
       value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
-      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
-      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
-      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
-      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+      uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
+      uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
+      uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
+      uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+      if constexpr (AFF) {  // integer levels -> scale * level + bias of each token
+        a0 = hfma2_bits(psab, a0, pbab);
+        a1 = hfma2_bits(psab, a1, pbab);
+        a2 = hfma2_bits(pscd, a2, pbcd);
+        a3 = hfma2_bits(pscd, a3, pbcd);
+      }
 #pragma unroll
       for (int j = 0; j < NT; ++j) mma16816(acc[j][mb], a0, a1, a2, a3, ppb[j][0], ppb[j][1]);
     }
@@ -632,47 +693,110 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
       load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
     }
+    uint32_t vsab = 0u, vbab = 0u, vscd = 0u, vbcd = 0u;
+    if constexpr (AFF) {
+      // the (scale, bias) words of this thread's value group for its four
+      // tokens; tokens past the end get (0, 0), so that their products with a
+      // zero probability stay zero whatever the staged bytes hold
+      const uint32_t* vm = reinterpret_cast<const uint32_t*>(st + Geo::offVN) + r0 * Geo::NG + (g * (D / 8)) / kAffineGroup;
+      const uint32_t ma = 2 * qd < n_valid ? vm[(2 * qd) * Geo::NG] : 0u;
+      const uint32_t mb = 2 * qd + 1 < n_valid ? vm[(2 * qd + 1) * Geo::NG] : 0u;
+      const uint32_t mc = 2 * qd + 8 < n_valid ? vm[(2 * qd + 8) * Geo::NG] : 0u;
+      const uint32_t md = 2 * qd + 9 < n_valid ? vm[(2 * qd + 9) * Geo::NG] : 0u;
+      vsab = __byte_perm(ma, mb, 0x5410);  // scales (low halves)
+      vbab = __byte_perm(ma, mb, 0x7632);  // biases (high halves)
+      vscd = __byte_perm(mc, md, 0x5410);
+      vbcd = __byte_perm(mc, md, 0x7632);
+    }
 
-    // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
-    // tokens g (hi/lo rows) and g + 8, each split over even / odd k-blocks so
-    // that the MMA accumulation chains are half as long
-    float sacc[2][NT][4], sacc2[2][NT][4];
+    float s0[NT], s1[NT];
+    if constexpr (!AFF) {
+      // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
+      // tokens g (hi/lo rows) and g + 8, each split over even / odd k-blocks so
+      // that the MMA accumulation chains are half as long
+      float sacc[2][NT][4], sacc2[2][NT][4];
 #pragma unroll
-    for (int par = 0; par < 2; ++par)
+      for (int par = 0; par < 2; ++par)
 #pragma unroll
-      for (int j = 0; j < NT; ++j)
+        for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[par][j][e] = sacc2[par][j][e] = 0.f;
-    {
-      uint32_t kw0[Geo::KW], kw1[Geo::KW];
-      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
-      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);  // bits of quarter qd, tokens g
-      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);  // and g + 8
+          for (int e = 0; e < 4; ++e) sacc[par][j][e] = sacc2[par][j][e] = 0.f;
+      {
+        uint32_t kw0[Geo::KW], kw1[Geo::KW];
+        const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
+        load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);  // bits of quarter qd, tokens g
+        load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);  // and g + 8
 #pragma unroll
-      for (int kb = 0; kb < Geo::KBLK; ++kb) {
-        const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
-        // one MMA per 8 tokens: rows g / g+8 carry token g's hi / lo key parts
-        const uint2 p0 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p1 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p2 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+        for (int kb = 0; kb < Geo::KBLK; ++kb) {
+          const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
+          // one MMA per 8 tokens: rows g / g+8 carry token g's hi / lo key parts
+          const uint2 p0 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+          const uint2 p1 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+          const uint2 p2 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+          const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          mma16816(sacc[kb & 1][j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
-          mma16816(sacc2[kb & 1][j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
+          for (int j = 0; j < NT; ++j) {
+            mma16816(sacc[kb & 1][j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
+            mma16816(sacc2[kb & 1][j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
+          }
         }
       }
-    }
-    const uint16_t* kn = reinterpret_cast<const uint16_t*>(st + Geo::offKN) + r0;
-    float s0[NT], s1[NT];
-    const float kn0 = __half2float(__ushort_as_half(kn[g])) * kpost;
-    const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
+      const uint16_t* kn = reinterpret_cast<const uint16_t*>(st + Geo::offKN) + r0;
+      const float kn0 = __half2float(__ushort_as_half(kn[g])) * kpost;
+      const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      s0[j] = (((sacc[0][j][0] + sacc[1][j][0]) + (sacc[0][j][1] + sacc[1][j][1])) +
-               ((sacc[0][j][2] + sacc[1][j][2]) + (sacc[0][j][3] + sacc[1][j][3]))) * kn0;
-      s1[j] = (((sacc2[0][j][0] + sacc2[1][j][0]) + (sacc2[0][j][1] + sacc2[1][j][1])) +
-               ((sacc2[0][j][2] + sacc2[1][j][2]) + (sacc2[0][j][3] + sacc2[1][j][3]))) * kn1;
+      for (int j = 0; j < NT; ++j) {
+        s0[j] = (((sacc[0][j][0] + sacc[1][j][0]) + (sacc[0][j][1] + sacc[1][j][1])) +
+                 ((sacc[0][j][2] + sacc[1][j][2]) + (sacc[0][j][3] + sacc[1][j][3]))) * kn0;
+        s1[j] = (((sacc2[0][j][0] + sacc2[1][j][0]) + (sacc2[0][j][1] + sacc2[1][j][1])) +
+                 ((sacc2[0][j][2] + sacc2[1][j][2]) + (sacc2[0][j][3] + sacc2[1][j][3]))) * kn1;
+      }
+    } else {
+      // ---- affine scores: rows g and g + 8 are two tokens (integer levels are
+      // exact in fp16); one accumulator per group, then
+      // s = sum_gg scale_gg * <levels, q>_gg + bias_gg * sum_gg(q)
+      float sacc[Geo::NG][NT][4];
+#pragma unroll
+      for (int gg = 0; gg < Geo::NG; ++gg)
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[gg][j][e] = 0.f;
+      uint32_t kw0[Geo::NG][Geo::KWA], kw1[Geo::NG][Geo::KWA];
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
+#pragma unroll
+      for (int gg = 0; gg < Geo::NG; ++gg) {
+        load_value_chunk<Geo::QBA, Geo::KWA, Geo::KNWA>(k0 + gg * 2 * KB, qd, kw0[gg]);
+        load_value_chunk<Geo::QBA, Geo::KWA, Geo::KNWA>(k0 + 8 * Geo::KS + gg * 2 * KB, qd, kw1[gg]);
+      }
+#pragma unroll
+      for (int kb = 0; kb < Geo::KBLK; ++kb) {
+        const int gg = kb >> 2, o1 = KB * 4 * (kb & 3), o2 = o1 + 2 * KB;
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane));
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(sacc[gg][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
+      }
+      const uint32_t* km = reinterpret_cast<const uint32_t*>(st + Geo::offKN) + r0 * Geo::NG;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) s0[j] = s1[j] = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < Geo::NG; ++gg) {
+        const float2 m0 = __half22float2(*reinterpret_cast<const __half2*>(km + g * Geo::NG + gg));
+        const float2 m1 = __half22float2(*reinterpret_cast<const __half2*>(km + (g + 8) * Geo::NG + gg));
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          s0[j] = fmaf(m0.x, sacc[gg][j][0] + sacc[gg][j][1], fmaf(m0.y, usc[j][gg], s0[j]));
+          s1[j] = fmaf(m1.x, sacc[gg][j][2] + sacc[gg][j][3], fmaf(m1.y, usc[j][gg], s1[j]));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        s0[j] *= kpost;
+        s1[j] *= kpost;
+      }
     }
     if constexpr (QJL) {
       float qacc[2][NT][4];
@@ -718,8 +842,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 
     // ---- online softmax (per warp, per head), P in fp16 hi/lo for the output MMA
     const uint16_t* vn = reinterpret_cast<const uint16_t*>(st + Geo::offVN) + r0;
-    const float vn0 = __half2float(__ushort_as_half(vn[g]));
-    const float vn1 = __half2float(__ushort_as_half(vn[g + 8]));
+    const float vn0 = AFF ? 1.f : __half2float(__ushort_as_half(vn[g]));
+    const float vn1 = AFF ? 1.f : __half2float(__ushort_as_half(vn[g + 8]));
     uint32_t pb[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
@@ -764,6 +888,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       ppb[j][0] = pb[j][0];
       ppb[j][1] = pb[j][1];
     }
+    psab = vsab;
+    pbab = vbab;
+    pscd = vscd;
+    pbcd = vbcd;
   }
   aggregate();  // the warp's last slab
 
@@ -902,22 +1030,22 @@ cudaError_t configure_kernel(KernelConfig& cfg, Kernel kern, int smem_bytes, int
 }
 
 // The decode kernel of one compile-time shape: configured, and its CTAs per SM.
-template <int D, int G, int KB, int VB, bool QJL>
+template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 cudaError_t configure_shape(int* ctas_per_sm) {
-  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
+  using Geo = DecodeGeom<D, G, KB, VB, QJL, AFF>;
   static KernelConfig cfg;  // one per shape
-  return configure_kernel(cfg, decode_kernel<D, G, KB, VB, QJL>, Geo::total, kDecThreads,
+  return configure_kernel(cfg, decode_kernel<D, G, KB, VB, QJL, AFF>, Geo::total, kDecThreads,
                           ctas_per_sm);
 }
 
 // Launches decode_kernel for one compile-time shape (grid: plan.ctas CTAs).
-template <int D, int G, int KB, int VB, bool QJL>
+template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const void* q, int dtype,
                                 int q_heads, float scale_log2, int max_ctx,
                                 const DecodePlan& plan, float* ws, cudaStream_t stream) {
-  using Geo = DecodeGeom<D, G, KB, VB, QJL>;
-  auto kern = decode_kernel<D, G, KB, VB, QJL>;
-  cudaError_t e = configure_shape<D, G, KB, VB, QJL>(nullptr);
+  using Geo = DecodeGeom<D, G, KB, VB, QJL, AFF>;
+  auto kern = decode_kernel<D, G, KB, VB, QJL, AFF>;
+  cudaError_t e = configure_shape<D, G, KB, VB, QJL, AFF>(nullptr);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.ctas);
@@ -933,16 +1061,17 @@ cudaError_t launch_decode_shape(const Tables& tb, const CacheView& cv, const voi
                             plan.slots, ws);
 }
 
-// Per-head-dim dispatch over (group, k_bits, v_bits, qjl); instantiated in the
-// tq_decode_d<D>.cu translation units.
-template <int D>
+// Per-head-dim, per-codec dispatch over (group, k_bits, v_bits, qjl);
+// instantiated in the tq_decode_d<D>.cu (Lloyd-Max) and tq_decode_affine_d<D>.cu
+// (affine) translation units.
+template <int D, bool AFF>
 cudaError_t decode_occupancy_dim(const Tables& tb, int group, int* ctas_per_sm);
 
-template <int D>
+template <int D, bool AFF>
 cudaError_t dispatch_occupancy_dim(const Tables& tb, int G, int* ctas_per_sm) {
 #define TQ_CASE(GG, KB, VB, QJ)                                             \
   if (G == GG && tb.k_bits == KB && tb.v_bits == VB && (tb.qjl != 0) == QJ) \
-    return configure_shape<D, GG, KB, VB, QJ>(ctas_per_sm);
+    return configure_shape<D, GG, KB, VB, QJ, AFF>(ctas_per_sm);
 #define TQ_BITS(GG, QJ) \
   TQ_CASE(GG, 2, 2, QJ) TQ_CASE(GG, 2, 3, QJ) TQ_CASE(GG, 3, 3, QJ) TQ_CASE(GG, 3, 4, QJ) TQ_CASE(GG, 4, 4, QJ)
 #define TQ_GROUP(GG) TQ_BITS(GG, false) TQ_BITS(GG, true)
@@ -956,20 +1085,20 @@ cudaError_t dispatch_occupancy_dim(const Tables& tb, int G, int* ctas_per_sm) {
   return cudaErrorNotSupported;
 }
 
-template <int D>
+template <int D, bool AFF>
 cudaError_t launch_decode_dim(const Tables& tb, const CacheView& cv, const void* q, int dtype,
                               int q_heads, float scale_log2, int max_ctx, const DecodePlan& plan,
                               float* ws, cudaStream_t stream);
 
-template <int D>
+template <int D, bool AFF>
 cudaError_t dispatch_decode_dim(const Tables& tb, const CacheView& cv, const void* q, int dtype,
                                 int q_heads, float scale_log2, int max_ctx,
                                 const DecodePlan& plan, float* ws, cudaStream_t stream) {
   const int G = q_heads / cv.kv_heads;
-#define TQ_CASE(GG, KB, VB, QJ)                                                               \
-  if (G == GG && tb.k_bits == KB && tb.v_bits == VB && (tb.qjl != 0) == QJ)                   \
-    return launch_decode_shape<D, GG, KB, VB, QJ>(tb, cv, q, dtype, q_heads, scale_log2,     \
-                                                  max_ctx, plan, ws, stream);
+#define TQ_CASE(GG, KB, VB, QJ)                                                                \
+  if (G == GG && tb.k_bits == KB && tb.v_bits == VB && (tb.qjl != 0) == QJ)                    \
+    return launch_decode_shape<D, GG, KB, VB, QJ, AFF>(tb, cv, q, dtype, q_heads, scale_log2, \
+                                                       max_ctx, plan, ws, stream);
 #define TQ_BITS(GG, QJ) \
   TQ_CASE(GG, 2, 2, QJ) TQ_CASE(GG, 2, 3, QJ) TQ_CASE(GG, 3, 3, QJ) TQ_CASE(GG, 3, 4, QJ) TQ_CASE(GG, 4, 4, QJ)
 #define TQ_GROUP(GG) TQ_BITS(GG, false) TQ_BITS(GG, true)

@@ -30,7 +30,12 @@ struct Tables {
   uint32_t s1[8];    // bit i set: channel i of D1 is -1
   uint32_t s2[8];    // same for D2 (QJL rotation)
   int d, k_bits, v_bits, qjl;
+  int affine;        // 1: the affine group-64 codec (centroids are the integer levels)
 };
+
+// Channels per group of the affine codec; its per-vector metadata is one
+// (scale, bias) fp16 pair, i.e. one 32-bit word, per group.
+constexpr int kAffineGroup = 64;
 
 struct CacheView {
   uint8_t *k_codes, *v_codes, *k_signs;

@@ -5,7 +5,9 @@
 //   keys with QJL: residual -> its norm -> second rotation -> sign bits.
 // ("TurboQuant Performance Benefits ...", "What Is TurboQuant?": random
 // Hadamard rotation then MSE codebook quantization; "mlx-turboquant" README,
-// "The 1-bit QJL residual": sign(RHT2(r)) and ||r||.)
+// "The 1-bit QJL residual": sign(RHT2(r)) and ||r||.)  The kernels are also
+// instantiated for the affine group-64 comparison codec (rotated keys, fp16
+// scale and bias per group of 64 channels: encode_affine_store).
 //
 // A group of d/32 adjacent lanes encodes one vector, each lane holding 32
 // consecutive channels, so a warp encodes 32*32/d vectors at once.  Five of
@@ -33,6 +35,31 @@ namespace {
 using namespace codec;
 
 constexpr int kAppendWarps = 8;
+
+// The codec of one vector at its code width: Lloyd-Max (norm, codes, sketch)
+// or the affine group-64 comparison codec (scale/bias pairs in `norm`).
+template <int D, int E, bool AFF>
+__device__ __forceinline__ void encode_vector(int bits, float (&u)[E], const Tables& tb, bool is_v,
+                                              int g, int lane, bool valid, uint8_t* codes,
+                                              uint16_t* norm, uint8_t* signs, uint16_t* rnorm,
+                                              const float* s_kcent, uint32_t* pack) {
+  if constexpr (AFF) {
+    uint32_t* meta = reinterpret_cast<uint32_t*>(norm);
+    if (bits == 2)
+      encode_affine_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+    else if (bits == 3)
+      encode_affine_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+    else
+      encode_affine_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+  } else {
+    if (bits == 2)
+      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    else if (bits == 3)
+      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    else
+      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+  }
+}
 constexpr int kAppendThreads = 32 * kAppendWarps;
 
 // Grid: (2 * blocks_per_kind, batch).  Blocks [0, blocks_per_kind) encode keys,
@@ -40,7 +67,7 @@ constexpr int kAppendThreads = 32 * kAppendWarps;
 // encodes one vector: E = 32 packs 32 * 32 / D vectors into a warp (throughput:
 // bulk appends); E = D / 32 gives each vector its own warp and keeps the
 // unrolled code short (latency: a few tokens per row, as in a decode step).
-template <int D, typename T, int E>
+template <int D, typename T, int E, bool AFF>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_append_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                            const T* __restrict__ kin, const T* __restrict__ vin, int n_new,
@@ -82,16 +109,14 @@ __global__ void __launch_bounds__(kAppendThreads)
     const long slot = ((long)b * cv.kv_heads + h) * cv.capacity + base + j;
     const int bits = is_v ? tb.v_bits : tb.k_bits;
     uint8_t* codes = (is_v ? cv.v_codes : cv.k_codes) + slot * (long)(bits * D / 8);
-    uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot;
+    // one fp16 norm per vector, or the affine codec's (scale, bias) per group
+    constexpr int NH = AFF ? 2 * D / kAffineGroup : 1;
+    uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
     uint32_t* pack = s_pack[tid >> 5];
-    if (bits == 2)
-      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
-    else if (bits == 3)
-      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
-    else
-      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent,
+                             pack);
   }
 
   // The last block of this batch row to finish publishes the new length.  Every
@@ -114,7 +139,7 @@ __global__ void __launch_bounds__(kAppendThreads)
 // smaller one (a [batch][T][heads][d] cache) and with h outermost otherwise,
 // so consecutive lanes read consecutive memory.  Without `lengths` every row
 // holds max_len vectors and no length or flag is written.
-template <int D, typename T, int E>
+template <int D, typename T, int E, bool AFF>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_convert_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                             const T* __restrict__ kin, const T* __restrict__ vin, long stride_b,
@@ -158,16 +183,14 @@ __global__ void __launch_bounds__(kAppendThreads)
     const long slot = ((long)b * H + h) * cv.capacity + t;
     const int bits = is_v ? tb.v_bits : tb.k_bits;
     uint8_t* codes = (is_v ? cv.v_codes : cv.k_codes) + slot * (long)(bits * D / 8);
-    uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot;
+    // one fp16 norm per vector, or the affine codec's (scale, bias) per group
+    constexpr int NH = AFF ? 2 * D / kAffineGroup : 1;
+    uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
     uint32_t* pack = s_pack[tid >> 5];
-    if (bits == 2)
-      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
-    else if (bits == 3)
-      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
-    else
-      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent,
+                             pack);
   }
   pdl_trigger();
 }
@@ -177,7 +200,7 @@ __global__ void __launch_bounds__(kAppendThreads)
 // latency rules; larger ones take the 32-channels-per-lane layout.
 constexpr long kLatencyVectors = 4096;
 
-template <int D, typename T, int E>
+template <int D, typename T, int E, bool AFF>
 cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                           int n_new, cudaStream_t stream) {
   constexpr int VPB = kAppendThreads / (D / E);
@@ -193,7 +216,7 @@ cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_append_kernel<D, T, E>, tb, cv,
+  return cudaLaunchKernelEx(&cfg, quantize_append_kernel<D, T, E, AFF>, tb, cv,
                             static_cast<const T*>(k), static_cast<const T*>(v), n_new,
                             (int)blocks_per_kind);
 }
@@ -202,11 +225,15 @@ template <int D, typename T>
 cudaError_t launch_typed(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                          int n_new, cudaStream_t stream) {
   const long vectors = 2L * cv.batch * cv.kv_heads * n_new;
-  if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32>(tb, cv, k, v, n_new, stream);
-  return launch_layout<D, T, 32>(tb, cv, k, v, n_new, stream);
+  if (tb.affine) {
+    if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, true>(tb, cv, k, v, n_new, stream);
+    return launch_layout<D, T, 32, true>(tb, cv, k, v, n_new, stream);
+  }
+  if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, false>(tb, cv, k, v, n_new, stream);
+  return launch_layout<D, T, 32, false>(tb, cv, k, v, n_new, stream);
 }
 
-template <int D, typename T, int E>
+template <int D, typename T, int E, bool AFF>
 cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const void* k,
                                   const void* v, long sb, long sh, long st,
                                   const int32_t* lengths, int max_len, int kinds,
@@ -224,7 +251,7 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_convert_kernel<D, T, E>, tb, cv,
+  return cudaLaunchKernelEx(&cfg, quantize_convert_kernel<D, T, E, AFF>, tb, cv,
                             static_cast<const T*>(k), static_cast<const T*>(v), sb, sh, st,
                             lengths, max_len, (int)blocks_per_kind, sh < st ? 1 : 0);
 }
@@ -234,10 +261,16 @@ cudaError_t launch_convert_typed(const Tables& tb, const CacheView& cv, const vo
                                  const void* v, long sb, long sh, long st, const int32_t* lengths,
                                  int max_len, int kinds, cudaStream_t stream) {
   const long vectors = (long)kinds * cv.batch * cv.kv_heads * max_len;
-  if (vectors <= kLatencyVectors)
-    return launch_convert_layout<D, T, D / 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds,
-                                               stream);
-  return launch_convert_layout<D, T, 32>(tb, cv, k, v, sb, sh, st, lengths, max_len, kinds, stream);
+  const bool small = vectors <= kLatencyVectors;
+  if (tb.affine)
+    return small ? launch_convert_layout<D, T, D / 32, true>(tb, cv, k, v, sb, sh, st, lengths,
+                                                             max_len, kinds, stream)
+                 : launch_convert_layout<D, T, 32, true>(tb, cv, k, v, sb, sh, st, lengths, max_len,
+                                                         kinds, stream);
+  return small ? launch_convert_layout<D, T, D / 32, false>(tb, cv, k, v, sb, sh, st, lengths,
+                                                            max_len, kinds, stream)
+               : launch_convert_layout<D, T, 32, false>(tb, cv, k, v, sb, sh, st, lengths, max_len,
+                                                        kinds, stream);
 }
 
 template <int D>
@@ -308,7 +341,7 @@ cudaError_t launch_quantize_cache(const Tables& tb, const CacheView& cv, const v
 cudaError_t launch_weights_quantize(const Tables& tb, const void* w, int dtype, int rows, int k,
                                     uint8_t* codes, uint16_t* norms, cudaStream_t stream) {
   Tables t = tb;
-  t.qjl = 0;  // weights carry only the MSE codes
+  t.qjl = 0;  // weights carry only the MSE codes (the API rejects the affine codec)
   CacheView cv = {};
   cv.k_codes = codes;  // block j of row n is "token" n of "head" j
   cv.k_norm = norms;

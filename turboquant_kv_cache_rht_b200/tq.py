@@ -38,12 +38,13 @@ class tq_params(C.Structure):
                 ("qjl", C.c_int), ("seed", C.c_uint64), ("codebook", C.c_int)]
 
 
-CODEBOOKS = {"gaussian": 0, "sphere": 1}   # TQ_CODEBOOK_GAUSSIAN, TQ_CODEBOOK_SPHERE
+# TQ_CODEBOOK_GAUSSIAN, TQ_CODEBOOK_SPHERE, TQ_CODEBOOK_AFFINE
+CODEBOOKS = {"gaussian": 0, "sphere": 1, "affine": 2}
 
 
 class tq_layout(C.Structure):
     _fields_ = [("k_code_bytes", C.c_size_t), ("v_code_bytes", C.c_size_t),
-                ("k_sign_bytes", C.c_size_t)]
+                ("k_sign_bytes", C.c_size_t), ("norm_halves", C.c_size_t)]
 
 
 class tq_cache(C.Structure):
@@ -117,8 +118,10 @@ class Codebook:
 
     def __init__(self, head_dim: int, k_bits: int, v_bits: int, qjl: bool = False, seed: int = 0,
                  codebook: str = "gaussian"):
-        """codebook: "gaussian" (Lloyd-Max for N(0,1)) or "sphere" (Lloyd-Max for
-        the exact distribution of a rotated coordinate, which depends on head_dim)."""
+        """codebook: "gaussian" (Lloyd-Max for N(0,1)), "sphere" (Lloyd-Max for
+        the exact distribution of a rotated coordinate, which depends on head_dim)
+        or "affine" (the affine group-64 comparison codec: rotated keys, fp16
+        scale and bias per group of 64 channels)."""
         if codebook not in CODEBOOKS:
             raise ValueError(f"codebook must be one of {sorted(CODEBOOKS)}")
         self.params = tq_params(head_dim, k_bits, v_bits, int(bool(qjl)), seed & ((1 << 64) - 1),
@@ -139,6 +142,7 @@ class Codebook:
     k_bits = property(lambda self: self.params.k_bits)
     v_bits = property(lambda self: self.params.v_bits)
     qjl = property(lambda self: bool(self.params.qjl))
+    affine = property(lambda self: self.params.codebook == CODEBOOKS["affine"])
 
     def tables(self) -> dict:
         """Host copies of the codebooks and rotation signs (tq_codebook_tables)."""
@@ -170,8 +174,10 @@ class Cache:
         self.k_codes = torch.zeros(*n, lay.k_code_bytes, **u8)
         self.v_codes = torch.zeros(*n, lay.v_code_bytes, **u8)
         self.k_signs = torch.zeros(*n, lay.k_sign_bytes, **u8) if cb.qjl else None
-        self.k_norm = torch.zeros(n, dtype=torch.float16, device=device)
-        self.v_norm = torch.zeros(n, dtype=torch.float16, device=device)
+        # one fp16 norm per vector, or (scale, bias) per group for the affine codec
+        nh = (lay.norm_halves,) if cb.affine else ()
+        self.k_norm = torch.zeros(*n, *nh, dtype=torch.float16, device=device)
+        self.v_norm = torch.zeros(*n, *nh, dtype=torch.float16, device=device)
         self.k_rnorm = torch.zeros(n, dtype=torch.float16, device=device) if cb.qjl else None
         self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)

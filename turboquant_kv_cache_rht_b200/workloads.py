@@ -40,6 +40,7 @@ class Workload:
     outlier_scale: float = 1.0
     corr_frac: float = 0.0          # fraction of key positions correlated with the query
     corr_cos: float = 0.0
+    codebook: str = "gaussian"      # "gaussian" | "sphere" | "affine" (the comparison codec)
     description: str = field(default="", compare=False)
 
     @property
@@ -69,6 +70,10 @@ WORKLOADS = {
                         ctx_range=(8192, 65536), outliers=4, outlier_scale=20.0,
                         description="batch 32, 32 q / 8 KV heads, d 128, ragged ctx U[8k, 64k], "
                                     "bf16, 3-bit K + 4-bit V, 1 appended token per step"),
+    "affine": Workload("affine", 1, 32, 8, 128, 4, 4, False, "bf16", 1006, context=32768,
+                       outliers=4, outlier_scale=20.0, codebook="affine",
+                       description="batch 1, 32 q / 8 KV heads, d 128, ctx 32768, bf16, affine "
+                                   "group-64 comparison codec: rotated 4-bit K + 4-bit V"),
 }
 
 
