@@ -57,6 +57,9 @@ DECODE_SOURCES = ("tq_internal.cuh", "tq_decode_impl.cuh", "tq_decode.cu", "tq_d
                   "tq_decode_affine_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
     "gqa": (31754240, "28c20c72a0cb8e28"),
+    "qjl": (566914304, "28c20c72a0cb8e28"),
+    "long": (353341952, "28c20c72a0cb8e28"),
+    "serving": (1102758656, "28c20c72a0cb8e28"),
     "affine": (38808064, "28c20c72a0cb8e28"),
 }
 
