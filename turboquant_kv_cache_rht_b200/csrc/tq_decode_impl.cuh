@@ -37,6 +37,15 @@
 // state; the four warps are merged in a fixed order and each segment's
 // partial (max, sum, output) goes to the workspace, where the combine kernel
 // merges the partials of every unit and applies the inverse rotation.
+//
+// AFF instantiates the same kernel for the affine group-64 comparison codec
+// ("mlx-turboquant" README, "Quantize the KV cache (long-context inference)",
+// "How it plugs in"): the tables hold the integer levels, a thread quarter
+// reads 16 channels of every 64-channel group (so each k-block lies in one
+// group), MMA rows g and g+8 are two tokens, the score sums
+// scale * <levels, q> + bias * sum(q) over the groups, values become
+// scale * level + bias by one hfma2 per operand pair, and nothing is rotated
+// back (values are stored unrotated).
 #pragma once
 
 #include "tq_internal.cuh"
