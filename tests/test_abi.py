@@ -221,3 +221,17 @@ def test_workspace_size_formula():
 def test_kv_bits_split_matches_oracle():
     for b in (2, 2.5, 3, 3.5, 4):
         assert tq.kv_bits_split(b) == o.kv_bits_split(b)
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa", "qjl", "long", "serving", "affine"])
+def test_bench_byte_model_matches_the_layout(name):
+    """bench.py's algorithmic bytes per stored (token, KV head) equal what the
+    library's layout says a decode must read: codes, the fp16 norm or (scale,
+    bias) words of K and V, and with QJL the sign plane plus an fp16 norm."""
+    import bench
+    from turboquant_kv_cache_rht_b200 import workloads as wl
+    w = wl.WORKLOADS[name]
+    lay = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, codebook=w.codebook).layout
+    per_token = (lay.k_code_bytes + lay.v_code_bytes + 2 * 2 * lay.norm_halves
+                 + ((lay.k_sign_bytes + 2) if w.qjl else 0))
+    assert bench.token_bytes(w) == per_token
