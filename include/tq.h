@@ -18,6 +18,9 @@
  *    inner-product estimator)": keys may carry sign(RHT2(r)) and ||r|| of the
  *    residual r = Rk - k_hat; the score adds
  *    sqrt(pi/(2d)) * ||r|| * <RHT2(Rq), sign(RHT2(r))>.
+ *  - same README, "Quantize the KV cache (long-context inference)" and "How
+ *    it plugs in": the affine group-64 cache with rotated keys, built here as
+ *    a comparison codec (TQ_CODEBOOK_AFFINE) on the same kernels.
  *
  * Conventions shared by every call:
  *  - Pointers are plain host or device addresses as stated per argument; the
