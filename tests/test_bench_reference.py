@@ -1,0 +1,41 @@
+"""The reference arm of bench.py (the oracle on the host cores), CPU only.
+
+Runs `bench.py --impl reference` on the small workloads and checks the JSON
+line the benchmark contract asks for: one line, the arm's own metric, unit
+and direction, a cpu_baseline describing the run, an e2e entry with no
+host-device copies, and a rejected warm-up below 3 steps.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*args):
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                          capture_output=True, text=True, timeout=600, cwd=ROOT)
+
+
+@pytest.mark.parametrize("workload", ["tiny", "affine"])
+def test_reference_arm_json_line(workload):
+    r = _run("--impl", "reference", "--workload", workload, "--steps", "3", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["steps"] == 3 and d["warmup"] == 3 and d["value"] > 0
+    assert d["config"]["workload"] == workload
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_warmup_below_three_is_rejected():
+    r = _run("--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "2")
+    assert r.returncode != 0 and "warmup" in r.stderr
