@@ -39,3 +39,21 @@ def test_reference_arm_json_line(workload):
 def test_warmup_below_three_is_rejected():
     r = _run("--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "2")
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_clock_summary_parses_nvidia_smi_lines():
+    """The clocks entry: median SM clock under load, max clock, active reasons."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.out = "\n".join([
+        "1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "1950, 1965, 900.3, 0x4, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 880.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ])
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    c.out = ""
+    assert c.summary()["reasons"] == ["unavailable"]
