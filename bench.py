@@ -1,8 +1,9 @@
 """Benchmark of the TurboQuant decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload gqa|qjl|long|serving|tiny|affine]
-                    [--impl ours|reference] [--no-dense] [--no-cpu-baseline] [--lutmm]
+                    [--workload serving|gqa|qjl|long|tiny|affine]
+                    [--impl ours|reference] [--no-dense] [--no-cpu-baseline]
+                    [--no-long-context] [--lutmm]
 
 A step is one pass of the whole hot path over one batch: tq_quantize_append of
 one new token per (batch row, KV head), then tq_decode_attention of every query
@@ -367,6 +368,12 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
 
     del graphs
     peak, peak_kind = peaks()
+    long_ctx = None
+    if world == 1 and not args.no_long_context:
+        del st.caches
+        torch.cuda.empty_cache()
+        long_ctx = {name: long_context_leg(name, dev, peak, dense=not args.no_dense)
+                    for name in ("qjl", "long") if name != w.name}
     achieved = dec_bytes / (dec_us * 1e-6) / 1e9
     hbm_frac = achieved / peak
     res = {
@@ -404,6 +411,30 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         res["dense_baseline"] = dense
     if lutmm is not None:
         res["lut_matmul"] = lutmm
+    if long_ctx:
+        res["long_context"] = long_ctx
+    return res
+
+
+def long_context_leg(name: str, dev, peak: float, dense: bool = True) -> dict:
+    """Decode-call time of one long-context workload (caches prefilled as in
+    the main leg, calls back to back over replicas > 4x L2), its fraction of
+    the HBM roofline, and the dense bf16 decode kernels on the same shape."""
+    w = wl.WORKLOADS[name]
+    st = State(w, 64, dev)
+    st_decode_us(st, dev, n=4)        # first calls configure the kernel of this shape
+    us = st_decode_us(st, dev, n=max(st.replicas, 16))
+    lens = [int(x) for x in st.caches[0].seq_lens.cpu()]
+    byts = step_bytes(w, lens)["decode"]
+    gbs = byts / (us * 1e-6) / 1e9
+    res = {"description": w.description, "decode_us": round(us, 2), "gb_s": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "ctx_tokens_per_s": round(sum(lens) / (us * 1e-6), 1),
+           "algorithmic_bytes_per_launch": byts}
+    if dense:
+        d = dense_baselines(w, st, dev)
+        res["dense_baseline"] = d
+    del st
+    torch.cuda.empty_cache()
     return res
 
 
@@ -700,10 +731,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="gqa", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="serving", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-long-context", action="store_true",
+                    help="skip the decode-call timing of the qjl and long workloads")
     ap.add_argument("--lutmm", action="store_true",
                     help="also time the weights-regime LUT matmul on a 16384 x 8192 layer")
     args = ap.parse_args()

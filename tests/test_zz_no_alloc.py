@@ -40,19 +40,26 @@ def _noalloc(cb, cache, q, out, max_ctx):
     return out
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
-    cb = tq.Codebook(128, 3, 4, qjl=True, seed=3)
+@pytest.mark.parametrize("d,kb,vb,qjl,codebook", [
+    (128, 3, 4, True, "gaussian"),     # the QJL sketch
+    (128, 3, 4, False, "gaussian"),
+    (128, 4, 4, False, "affine"),      # the affine comparison codec
+    (256, 2, 2, True, "gaussian"),     # head_dim 256, 2-bit codes
+])
+def test_noalloc_matches_workspace_entry_point_twice(d, kb, vb, qjl, codebook):
+    cb = tq.Codebook(d, kb, vb, qjl=qjl, seed=3, codebook=codebook)
     cases = [(2, 4, 4, 1000, 1024, 11), (1, 8, 2, 3000, 3008, 12)]   # two calls in a row
     for batch, kv_heads, group, length, cap, seed in cases:
+        assert tq.tq_decode_workspace_bytes(cb, batch, kv_heads * group, kv_heads, cap) <= (8 << 20)
         cache = _filled_cache(cb, batch, kv_heads, length, cap, seed)
         g = torch.Generator().manual_seed(seed + 100)
-        q = torch.randn(batch, kv_heads * group, 128, generator=g).bfloat16().cuda()
-        out = torch.full((batch, kv_heads * group, 128), float("nan"), device="cuda")
+        q = torch.randn(batch, kv_heads * group, d, generator=g).bfloat16().cuda()
+        out = torch.full((batch, kv_heads * group, d), float("nan"), device="cuda")
         got = _noalloc(cb, cache, q, out, cap).clone()
         ref = tq.tq_decode_attention(cb, cache, q, max_ctx=cap)
         torch.cuda.synchronize()
         assert torch.isfinite(got).all()
-        assert_rows_close(got.cpu().numpy().reshape(-1, 128), ref.cpu().numpy().reshape(-1, 128))
+        assert_rows_close(got.cpu().numpy().reshape(-1, d), ref.cpu().numpy().reshape(-1, d))
 
 
 def test_noalloc_rejects_decodes_larger_than_its_scratch():

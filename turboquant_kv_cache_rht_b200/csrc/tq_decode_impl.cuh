@@ -148,6 +148,12 @@ __device__ __forceinline__ uint32_t hfma2_bits(uint32_t s, uint32_t c, uint32_t 
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// a * b on half2 bit patterns
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // +-1.0 half2 from the two sign bits at positions 15 and 31 (bit 1 -> +1)
 __device__ __forceinline__ uint32_t sign_pair(uint32_t x) { return (x & 0x80008000u) ^ 0xBC00BC00u; }
 
@@ -849,16 +855,48 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     }
     const bool ok0 = g < n_valid, ok1 = g + 8 < n_valid;
 
+    // ---- value magnitude of tokens g, g + 8 as a power of two 2^ev (ev an
+    //      integer) and the factor m = |v| 2^-ev in [0, 2) that stays with the
+    //      weight.  The running maximum below is taken over s + ev, so every
+    //      weight p * |v| = 2^(s - max) |v| <= 2^-ev |v| < 2 lies in fp16's
+    //      normal range whatever the norms are (tiny, huge or mixed), and the
+    //      hi/lo split of P keeps its ~22 bits.  Lloyd-Max: |v| is the stored
+    //      fp16 norm, ev its exponent (subnormals and zero as 2^-14).  Affine:
+    //      ev is the exponent of the token's largest |scale| or |bias| (clamped
+    //      to [-14, 14]); the value side scales (scale, bias) by 2^-ev exactly.
+    float vm0, vm1, ev0, ev1;
+    uint32_t vfac = 0u;  // affine: fp16 bits of 2^-ev of tokens g (low) and g + 8 (high)
+    if constexpr (!AFF) {
+      const uint16_t* vn = reinterpret_cast<const uint16_t*>(st + Geo::offVN) + r0;
+      const uint32_t b0 = vn[g], b1 = vn[g + 8];
+      vm0 = __half2float(__ushort_as_half((uint16_t)b0));
+      vm1 = __half2float(__ushort_as_half((uint16_t)b1));
+      ev0 = (float)(max((int)((b0 >> 10) & 31u), 1) - 15);
+      ev1 = (float)(max((int)((b1 >> 10) & 31u), 1) - 15);
+    } else {
+      const uint32_t* vmw = reinterpret_cast<const uint32_t*>(st + Geo::offVN) + (r0 + g) * Geo::NG;
+      uint32_t f0 = 1u, f1 = 1u;  // largest fp16 exponent field among |scale|, |bias|
+#pragma unroll
+      for (int gg = 0; gg < Geo::NG; ++gg) {
+        const uint32_t x0 = vmw[gg], x1 = vmw[8 * Geo::NG + gg];
+        f0 = max(f0, max((x0 >> 10) & 31u, (x0 >> 26) & 31u));
+        f1 = max(f1, max((x1 >> 10) & 31u, (x1 >> 26) & 31u));
+      }
+      const int e0 = min((int)f0, 29) - 15, e1 = min((int)f1, 29) - 15;  // [-14, 14]
+      ev0 = (float)e0;
+      ev1 = (float)e1;
+      vm0 = __int_as_float((e0 + 127) << 23);  // 2^ev exactly
+      vm1 = __int_as_float((e1 + 127) << 23);
+      vfac = (uint32_t)((15 - e0) << 10) | ((uint32_t)((15 - e1) << 10) << 16);
+    }
+
     // ---- online softmax (per warp, per head), P in fp16 hi/lo for the output MMA
-    const uint16_t* vn = reinterpret_cast<const uint16_t*>(st + Geo::offVN) + r0;
-    const float vn0 = AFF ? 1.f : __half2float(__ushort_as_half(vn[g]));
-    const float vn1 = AFF ? 1.f : __half2float(__ushort_as_half(vn[g + 8]));
     uint32_t pb[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       if (!ok0) s0[j] = -INFINITY;
       if (!ok1) s1[j] = -INFINITY;
-      float mx = fmaxf(s0[j], s1[j]);
+      float mx = fmaxf(s0[j] + ev0, s1[j] + ev1);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -874,7 +912,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       const float p0 = ok0 ? fast_exp2(s0[j] - m_run[j]) : 0.f;
       const float p1 = ok1 ? fast_exp2(s1[j] - m_run[j]) : 0.f;
       l_part[j] += p0 + p1;
-      const float w0 = ok0 ? p0 * vn0 : 0.f, w1 = ok1 ? p1 * vn1 : 0.f;
+      const float w0 = ok0 ? p0 * vm0 : 0.f, w1 = ok1 ? p1 * vm1 : 0.f;
       uint32_t whi, wlo;
       split_pair(w0, w1, whi, wlo);
       const uint32_t x1h = __shfl_sync(0xffffffffu, whi, src1), x1l = __shfl_sync(0xffffffffu, wlo, src1);
@@ -897,10 +935,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       ppb[j][0] = pb[j][0];
       ppb[j][1] = pb[j][1];
     }
-    psab = vsab;
-    pbab = vbab;
-    pscd = vscd;
-    pbcd = vbcd;
+    if constexpr (AFF) {
+      // (scale, bias) of tokens 2q, 2q+1 and 2q+8, 2q+9 times their 2^-ev
+      // (exact: powers of two), from the lanes that scored those tokens
+      const uint32_t x1 = __shfl_sync(0xffffffffu, vfac, src1), x2 = __shfl_sync(0xffffffffu, vfac, src2);
+      const uint32_t fab = __byte_perm(x1, x2, 0x5410), fcd = __byte_perm(x1, x2, 0x7632);
+      psab = hmul2_bits(vsab, fab);
+      pbab = hmul2_bits(vbab, fab);
+      pscd = hmul2_bits(vscd, fcd);
+      pbcd = hmul2_bits(vbcd, fcd);
+    }
   }
   aggregate();  // the warp's last slab
 
