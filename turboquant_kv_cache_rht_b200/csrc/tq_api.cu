@@ -188,6 +188,40 @@ bool build_codebook(int bits, int kind, int d, float* cent, float* bnd) {
   return true;
 }
 
+// fp16 rounding of a float in fp16's normal range, to nearest even (the
+// table scale search below only meets magnitudes in [2^-14, 2^15)).
+double round_fp16_normal(float x) {
+  int e = 0;
+  const double m = std::frexp((double)x, &e);       // x = m 2^e, 0.5 <= |m| < 1
+  return std::ldexp(std::nearbyint(std::ldexp(m, 11)), e - 11);  // 11 significant bits
+}
+
+// Scale lam in [1, 2) under which the fp16 roundings of lam * c_j (formed as
+// an fp32 product, as the decode kernel forms it) come closest to the exact
+// products: the largest relative rounding error over the nonzero entries is
+// minimal.  The decode kernel's code tables hold fp16(lam * c_j) and undo lam
+// in fp32, so a table of 4, 8 or 16 Lloyd-Max levels carries ~2^-22, ~2^-16
+// or ~2^-13 relative error instead of fp16's 2^-12.
+float fp16_table_scale(const float* cent, int levels) {
+  constexpr int kSteps = 1 << 16;
+  float best = 1.0f;
+  double best_err = INFINITY;
+  for (int i = 0; i < kSteps; ++i) {
+    const float lam = 1.0f + (float)i / (float)kSteps;
+    double err = 0.0;
+    for (int j = levels / 2; j < levels && err < best_err; ++j) {  // odd symmetry
+      const float x = cent[j] * lam;
+      if (x == 0.0f) continue;
+      err = std::max(err, std::fabs(round_fp16_normal(x) - (double)x) / std::fabs((double)x));
+    }
+    if (err < best_err) {
+      best_err = err;
+      best = lam;
+    }
+  }
+  return best;
+}
+
 // Affine codec tables: the integer levels 0 .. 2^bits - 1 and their midpoints
 // (the decode kernel's pair tables turn code pairs into these levels).
 void build_affine_levels(int bits, float* cent, float* bnd) {
@@ -315,6 +349,8 @@ tq_status tq_codebook_init(const tq_params* params, tq_codebook** out, tq_layout
     delete cb;
     return fail(TQ_ERR_INVALID, "Lloyd-Max iteration did not converge");
   }
+  t.k_lam = t.affine ? 1.0f : fp16_table_scale(t.k_cent, 1 << params->k_bits);
+  t.v_lam = t.affine ? 1.0f : fp16_table_scale(t.v_cent, 1 << params->v_bits);
   build_signs(params->seed, params->head_dim, t.s1);
   build_signs(params->seed ^ 0x9E3779B97F4A7C15ull, params->head_dim, t.s2);
   if (layout) {

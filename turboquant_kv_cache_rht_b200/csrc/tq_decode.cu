@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (int e = 0; e < E; ++e) part[warp][lane * E + e] = a[e];
   __syncthreads();
   if (warp == 0) {
-    const float inv = 1.0f / (tb.affine ? l : l * (float)D);
+    const float inv = 1.0f / (tb.affine ? l : l * (float)D * tb.v_lam);
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {

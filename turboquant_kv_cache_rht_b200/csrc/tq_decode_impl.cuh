@@ -61,6 +61,7 @@ constexpr int kDecWarps = 4;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kDecTile = 16 * kDecWarps;  // tokens per pipeline stage
 constexpr int kDecStages = 3;
+constexpr float kLazyLog2 = 8.0f;  // online-softmax slack before a rescale (log2 units)
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -208,13 +209,13 @@ struct DecodeGeom {
   static constexpr int VCH = VB * D / 8;      // value bits per thread group
   static constexpr int VCW = (VCH + 31) / 32; // words of the aligned value chunk
   static constexpr int VNW = (VCH % 32 == 0) ? VCH / 32 : (VCH + 16 + 31) / 32;
-  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (8 bytes: hi pair, lo pair)
+  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (4 bytes: an fp16 pair)
   static constexpr int LV = 1 << (2 * VB);    // value pair-table entries (4 bytes each)
   // Each table is replicated so that lanes with different (lane mod copies)
-  // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * size.
-  static constexpr int RKL = KB <= 3 ? 4 : 3;  // log2 key copies (16 or 8)
+  // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * 4.
+  static constexpr int RKL = KB <= 3 ? 5 : 4;  // log2 key copies (32 or 16)
   static constexpr int RVL = VB <= 3 ? 5 : 4;  // log2 value copies (32 or 16)
-  static constexpr int KSH = 3 + RKL;          // byte shift of a key entry index (8-byte entries)
+  static constexpr int KSH = 2 + RKL;          // byte shift of a key entry index
   static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
   // affine codec: NG groups of 64 channels, one (scale, bias) word per group
   // and token; thread quarter qd reads channels [64 gg + 16 qd, + 16) of group gg
@@ -238,7 +239,7 @@ struct DecodeGeom {
       (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
   // after the stage area
   static constexpr int offLK = stagesBytes;
-  static constexpr int offLV = offLK + (LK << RKL) * 8;
+  static constexpr int offLV = offLK + (LK << RKL) * 4;
   static constexpr int offQ = offLV + (LV << RVL) * 4;         // float [G][D] rotated query
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
@@ -379,25 +380,24 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, qd = lane & 3;
   const int H = cv.kv_heads;
-  // ---- pair tables: keys (hi pair, lo pair), values (fp16 pair).  They
-  //      depend on the kernel parameters alone, so they are built before the
-  //      wait, overlapping the previous kernel in the stream.
+  // ---- pair tables (two codes -> an fp16 pair) of the keys and of the
+  //      values, each centroid scaled by its table's k_lam / v_lam so that
+  //      its fp16 rounding is nearly exact.  They depend on the kernel
+  //      parameters alone, so they are built before the wait, overlapping the
+  //      previous kernel in the stream.
   {
     // each entry is computed once and written to all its copies with 16-byte stores
     constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
     for (int p = tid; p < Geo::LK; p += kDecThreads) {
-      const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
-      const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
-      const __half la = __float2half_rn(ca - __half2float(ha));
-      const __half lb = __float2half_rn(cb - __half2float(hb));
-      const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 2);
+      const uint32_t k = pack_half2(__float2half_rn(tb.k_cent[p & ((1 << KB) - 1)] * tb.k_lam),
+                                    __float2half_rn(tb.k_cent[p >> KB] * tb.k_lam));
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 4);
 #pragma unroll
-      for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(hi, lo, hi, lo);
+      for (int c = 0; c < RK / 4; ++c) dst[c] = make_uint4(k, k, k, k);
     }
     for (int p = tid; p < Geo::LV; p += kDecThreads) {
-      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)]),
-                                    __float2half_rn(tb.v_cent[p >> VB]));
+      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)] * tb.v_lam),
+                                    __float2half_rn(tb.v_cent[p >> VB] * tb.v_lam));
       uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * (RV / 4);
 #pragma unroll
       for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   // softmax scale, log2(e), the rotation's and the dequantization's 1/sqrt(d)
   // (and sqrt(pi/(2d)) of the QJL estimate)
   // (affine: the keys are in the orthonormal frame, only the query's H is unnormalized)
-  const float kpost = AFF ? scale_log2 / (sqrtf((float)D) * qsc) : scale_log2 / ((float)D * qsc);
+  const float kpost = AFF ? scale_log2 / (sqrtf((float)D) * qsc) : scale_log2 / ((float)D * qsc * tb.k_lam);
   const float qpost = scale_log2 * sqrtf(3.14159265358979f / (2.0f * D)) / ((float)D * qsc2);
 
   // ---- B fragments (query columns) in registers
@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   }
   const uint8_t* lutK = smem + Geo::offLK;
   const uint8_t* lutV = smem + Geo::offLV;
-  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 3;
+  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 2;
   const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
   const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
 
@@ -726,16 +726,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 
     float s0[NT], s1[NT];
     if constexpr (!AFF) {
-      // ---- scores: S = K_hat . Qt on the tensor cores, keys as hi + lo
-      // tokens g (hi/lo rows) and g + 8, each split over even / odd k-blocks so
-      // that the MMA accumulation chains are half as long
-      float sacc[2][NT][4], sacc2[2][NT][4];
+      // ---- scores: S = K_hat . Qt on the tensor cores; MMA rows g and g + 8
+      // are tokens g and g + 8, each k-block split over even / odd
+      // accumulators so that the MMA accumulation chains are half as long
+      float sacc[2][NT][4];
 #pragma unroll
       for (int par = 0; par < 2; ++par)
 #pragma unroll
         for (int j = 0; j < NT; ++j)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[par][j][e] = sacc2[par][j][e] = 0.f;
+          for (int e = 0; e < 4; ++e) sacc[par][j][e] = 0.f;
       {
         uint32_t kw0[Geo::KW], kw1[Geo::KW];
         const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
@@ -744,16 +744,12 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
         for (int kb = 0; kb < Geo::KBLK; ++kb) {
           const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
-          // one MMA per 8 tokens: rows g / g+8 carry token g's hi / lo key parts
-          const uint2 p0 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-          const uint2 p1 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
-          const uint2 p2 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-          const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            mma16816(sacc[kb & 1][j], p0.x, p0.y, p1.x, p1.y, bk[j][kb][0], bk[j][kb][1]);
-            mma16816(sacc2[kb & 1][j], p2.x, p2.y, p3.x, p3.y, bk[j][kb][0], bk[j][kb][1]);
-          }
+          for (int j = 0; j < NT; ++j) mma16816(sacc[kb & 1][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
         }
       }
       const uint16_t* kn = reinterpret_cast<const uint16_t*>(st + Geo::offKN) + r0;
@@ -761,10 +757,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       const float kn1 = __half2float(__ushort_as_half(kn[g + 8])) * kpost;
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        s0[j] = (((sacc[0][j][0] + sacc[1][j][0]) + (sacc[0][j][1] + sacc[1][j][1])) +
-                 ((sacc[0][j][2] + sacc[1][j][2]) + (sacc[0][j][3] + sacc[1][j][3]))) * kn0;
-        s1[j] = (((sacc2[0][j][0] + sacc2[1][j][0]) + (sacc2[0][j][1] + sacc2[1][j][1])) +
-                 ((sacc2[0][j][2] + sacc2[1][j][2]) + (sacc2[0][j][3] + sacc2[1][j][3]))) * kn1;
+        s0[j] = ((sacc[0][j][0] + sacc[0][j][1]) + (sacc[1][j][0] + sacc[1][j][1])) * kn0;
+        s1[j] = ((sacc[0][j][2] + sacc[0][j][3]) + (sacc[1][j][2] + sacc[1][j][3])) * kn1;
       }
     } else {
       // ---- affine scores: rows g and g + 8 are two tokens (integer levels are
@@ -900,14 +894,19 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      if (mx > m_run[j]) {
-        const float alpha = fast_exp2(m_run[j] - mx);
+      // lazy rescale: the running maximum moves only when a score passes it by
+      // more than kLazyLog2, so p stays below 2^kLazyLog2 and the weights below
+      // 2^(kLazyLog2 + 1) (well inside fp16); the vote keeps the branch uniform
+      // and, after the first slabs, almost never taken
+      if (__any_sync(0xffffffffu, mx > m_run[j] + kLazyLog2)) {
+        const float mn = fmaxf(m_run[j], mx);
+        const float alpha = fast_exp2(m_run[j] - mn);
         l_part[j] *= alpha;
 #pragma unroll
         for (int mb = 0; mb < Geo::MBLK; ++mb)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[j][mb][e] *= alpha;
-        m_run[j] = mx;
+        m_run[j] = mn;
       }
       const float p0 = ok0 ? fast_exp2(s0[j] - m_run[j]) : 0.f;
       const float p1 = ok1 ? fast_exp2(s1[j] - m_run[j]) : 0.f;

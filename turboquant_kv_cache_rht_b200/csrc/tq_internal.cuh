@@ -31,6 +31,11 @@ struct Tables {
   uint32_t s2[8];    // same for D2 (QJL rotation)
   int d, k_bits, v_bits, qjl;
   int affine;        // 1: the affine group-64 codec (centroids are the integer levels)
+  // Scales in [1, 2) of the decode kernel's fp16 code tables: they hold
+  // fp16(k_lam * k_cent[j]) and fp16(v_lam * v_cent[j]), chosen so that these
+  // roundings are nearly exact; the kernels divide the scale out in fp32
+  // (1 for the affine codec, whose levels are small integers).
+  float k_lam, v_lam;
 };
 
 // Channels per group of the affine codec; its per-vector metadata is one
