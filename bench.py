@@ -681,7 +681,7 @@ class OracleUnit:
         return (self.T + 1) * token_bytes(w) + w.group * d * (esz + 4) + 2 * d * esz + vec_out
 
 
-def cpu_baseline(w: wl.Workload, budget_s: float = 12.0) -> dict:
+def cpu_baseline(w: wl.Workload, budget_s: float = 10.0) -> dict:
     u = OracleUnit(w)
     u.step()
     t0 = time.perf_counter()
@@ -692,11 +692,46 @@ def cpu_baseline(w: wl.Workload, budget_s: float = 12.0) -> dict:
         el = time.perf_counter() - t0
         if el > budget_s or n >= 200:
             break
-    return {"value": round(n * u.bytes_per_step() / el / 1e9, 4), "unit": "GB/s",
-            "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} steps of one (batch row, KV head) unit: encode 1 appended K and V, "
-                      f"decode {w.group} query heads over {u.T + 1} tokens (numpy, float64 attention)",
-            "host_cpus": os.cpu_count()}
+    res = {"value": round(n * u.bytes_per_step() / el / 1e9, 4), "unit": "GB/s",
+           "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{n} steps of one (batch row, KV head) unit: encode 1 appended K and V, "
+                     f"decode {w.group} query heads over {u.T + 1} tokens (numpy, float64 attention)",
+           "host_cpus": os.cpu_count()}
+    res.update(oracle_rates(u))
+    return res
+
+
+def oracle_rates(u: "OracleUnit", budget_s: float = 2.0) -> dict:
+    """The oracle's quantize rate (Mvec/s: K and V vectors, keys with the QJL
+    sketch when the workload has it) and decode rate (ctx-tokens/s of one KV
+    head's G query heads), on all BLAS threads and on one thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        threadpool_limits = None
+    w = u.w
+    k, v = wl.kv_unit(w, 0, 0, 1024)
+    kf, vf = k.float().numpy(), v.float().numpy()
+
+    def rate(fn, units):
+        fn()
+        t0, n = time.perf_counter(), 0
+        while True:
+            fn()
+            n += 1
+            el = time.perf_counter() - t0
+            if el > budget_s:
+                return n * units / el
+
+    def measure():
+        return {"quantize_mvec_s": round(rate(lambda: u._encode(kf, vf), 2 * len(kf)) / 1e6, 5),
+                "decode_ctx_tokens_s": round(rate(u.step, u.T + 1), 1)}
+
+    out = {"all_threads": measure()}
+    if threadpool_limits is not None:
+        with threadpool_limits(limits=1):
+            out["one_thread"] = measure()
+    return out
 
 
 def run_reference(args, rank: int) -> dict | None:
