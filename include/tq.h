@@ -59,6 +59,8 @@ typedef enum {
 /* Sticky device-side flags ORed into *tq_cache.status. */
 #define TQ_FLAG_CAPACITY 1u  /* an append would pass `capacity`: that batch row was skipped */
 #define TQ_FLAG_MAXCTX 2u    /* a sequence was longer than the decode's max_ctx: its tail was not attended */
+#define TQ_FLAG_LAYOUT 4u    /* the decode kernel found its shared memory placed other than the host
+                                checked (never expected on sm_100a): its outputs are not valid */
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 

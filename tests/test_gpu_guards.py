@@ -127,6 +127,7 @@ def test_append_and_decode_stay_in_bounds(d, kb, vb, qjl, codebook):
         assert torch.all(out[2] == 0)
         flagged = bool(int(cache.status.item()) & tq.TQ_FLAG_MAXCTX)
         assert flagged == (max_ctx < cap)
+        assert not int(cache.status.item()) & tq.TQ_FLAG_LAYOUT
 
 
 @pytest.mark.parametrize("d,kb,vb,qjl,codebook", SHAPES[:5] + SHAPES[6:7])

@@ -119,6 +119,29 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// log2(x) with the hardware approximation (x > 0 here).
+__device__ __forceinline__ float fast_log2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-window address at which the dynamic shared memory of the decode
+// kernel starts: after the 1 KB the hardware reserves per CTA (the kernel
+// declares no static shared memory).  The host checks both facts before the
+// first launch and the kernel checks the address on entry.
+constexpr uint32_t kDynSmemBase = 0x400;
+
+// 32-bit load from a code table at shared-window address OFF + idx: the
+// table's address is an immediate of the load, so a lookup costs the index
+// arithmetic alone.
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds_table(uint32_t idx) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(idx), "n"(OFF));
+  return v;
+}
+
 // (a, b) -> half2 of their fp16 roundings (hi) and of the remainders (lo).
 __device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -213,8 +236,10 @@ struct DecodeGeom {
   static constexpr int LV = 1 << (2 * VB);    // value pair-table entries (4 bytes each)
   // Each table is replicated so that lanes with different (lane mod copies)
   // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * 4.
-  static constexpr int RKL = KB <= 3 ? 5 : 4;  // log2 key copies (32 or 16)
-  static constexpr int RVL = VB <= 3 ? 5 : 4;  // log2 value copies (32 or 16)
+  // 32 copies (a lane's own) keep every lookup free of bank conflicts; the
+  // 4-bit tables of head_dim 256 keep 16 to leave room for the stages
+  static constexpr int RKL = (KB <= 3 || D <= 128) ? 5 : 4;  // log2 key copies
+  static constexpr int RVL = (VB <= 3 || D <= 128) ? 5 : 4;  // log2 value copies
   static constexpr int KSH = 2 + RKL;          // byte shift of a key entry index
   static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
   // affine codec: NG groups of 64 channels, one (scale, bias) word per group
@@ -244,7 +269,9 @@ struct DecodeGeom {
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
   static constexpr int offRed = offUs + (AFF ? (G * NG * 4 + 15) / 16 * 16 : 0);  // float scratch
-  static constexpr int redFloats = (16 > 5 * G ? 16 : 5 * G) + 16;
+  // prologue: per-warp query maxima [2 * warps]; epilogue: merge weights
+  // [warps][G] then the group maxima [G]
+  static constexpr int redFloats = (2 * kDecWarps > (kDecWarps + 1) * G ? 2 * kDecWarps : (kDecWarps + 1) * G) + 16;
   // work schedule: scan scratch (one 64-bit word per warp), then one chunk of
   // rows (index, 64-bit tile prefix)
   static constexpr int offSched = (offRed + redFloats * 4 + 15) / 16 * 16;
@@ -362,11 +389,12 @@ __device__ __forceinline__ long long block_exclusive_scan(long long x, long long
   return before + inc - x;
 }
 
-// CTAs per SM the register budget is sized for: d <= 128 fits four CTAs (128
-// registers) unless the shape carries two column tiles or the QJL sketch,
-// which need up to 168 registers (three CTAs); d = 256 fits two.
+// CTAs per SM the register budget is sized for: d <= 128 fits three CTAs
+// (168 registers: measured faster than four CTAs at 128, where the kernel
+// spends instructions on register moves), two when the shape carries two
+// column tiles and the QJL sketch; d = 256 fits two.
 template <int D, int G, bool QJL>
-constexpr int decode_min_ctas() { return D <= 128 ? ((G > 4 || QJL) ? 3 : 4) : 2; }
+constexpr int decode_min_ctas() { return D <= 128 ? ((G > 4 && QJL) ? 2 : 3) : 2; }
 
 template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
@@ -380,6 +408,12 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, qd = lane & 3;
   const int H = cv.kv_heads;
+  // the code-table lookups address shared memory by immediates that assume
+  // where the dynamic shared memory starts (checked on the host as well)
+  if ((uint32_t)__cvta_generic_to_shared(smem) != kDynSmemBase) {
+    if (tid == 0) atomicOr(cv.status, (int)kFlagLayout);
+    return;
+  }
   // ---- pair tables (two codes -> an fp16 pair) of the keys and of the
   //      values, each centroid scaled by its table's k_lam / v_lam so that
   //      its fp16 rounding is nearly exact.  They depend on the kernel
@@ -498,7 +532,9 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
         cp_async16(st + Geo::offRN + tid * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + tid * 16);
     } else {
       // norms: rows * 2 bytes each = rows / 8 chunks per array
-      const int c = tid & 7, arr = tid >> 3;
+      constexpr int NC = kDecTile / 8;  // 16-byte chunks of one norm array in a full tile
+      static_assert(3 * NC <= kDecThreads, "one thread per norm chunk");
+      const int c = tid % NC, arr = tid / NC;
       if (c < rows / 8) {
         if (arr == 0)
           cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
@@ -573,11 +609,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   }
   if (lane == 0) {
     red[warp] = amax;
-    red[8 + warp] = amax2;
+    red[kDecWarps + warp] = amax2;
   }
   __syncthreads();
-  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  amax2 = fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
+  amax = red[0];
+  amax2 = red[kDecWarps];
+#pragma unroll
+  for (int w = 1; w < kDecWarps; ++w) {
+    amax = fmaxf(amax, red[w]);
+    amax2 = fmaxf(amax2, red[kDecWarps + w]);
+  }
   int e1 = 0, e2 = 0;
   frexpf(amax > 0.f ? amax : 1.f, &e1);
   frexpf(amax2 > 0.f ? amax2 : 1.f, &e2);
@@ -646,8 +687,6 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mb][e] = 0.f;
   }
-  const uint8_t* lutK = smem + Geo::offLK;
-  const uint8_t* lutV = smem + Geo::offLV;
   const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 2;
   const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
   const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
@@ -671,10 +710,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       uint32_t e0, o0, e1, o1;
       value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
       value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
-      uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutV + e0);
-      uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutV + o0);
-      uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutV + e1);
-      uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutV + o1);
+      uint32_t a0 = lds_table<kDynSmemBase + Geo::offLV>(e0);
+      uint32_t a1 = lds_table<kDynSmemBase + Geo::offLV>(o0);
+      uint32_t a2 = lds_table<kDynSmemBase + Geo::offLV>(e1);
+      uint32_t a3 = lds_table<kDynSmemBase + Geo::offLV>(o1);
       if constexpr (AFF) {  // integer levels -> scale * level + bias of each token
         a0 = hfma2_bits(psab, a0, pbab);
         a1 = hfma2_bits(psab, a1, pbab);
@@ -744,10 +783,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
         for (int kb = 0; kb < Geo::KBLK; ++kb) {
           const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
-          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
-          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+          const uint32_t a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+          const uint32_t a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+          const uint32_t a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+          const uint32_t a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
 #pragma unroll
           for (int j = 0; j < NT; ++j) mma16816(sacc[kb & 1][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
         }
@@ -781,10 +820,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int gg = kb >> 2, o1 = KB * 4 * (kb & 3), o2 = o1 + 2 * KB;
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
+        const uint32_t a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
+        const uint32_t a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
+        const uint32_t a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma16816(sacc[gg][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
       }
@@ -849,15 +888,15 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     }
     const bool ok0 = g < n_valid, ok1 = g + 8 < n_valid;
 
-    // ---- value magnitude of tokens g, g + 8 as a power of two 2^ev (ev an
-    //      integer) and the factor m = |v| 2^-ev in [0, 2) that stays with the
-    //      weight.  The running maximum below is taken over s + ev, so every
-    //      weight p * |v| = 2^(s - max) |v| <= 2^-ev |v| < 2 lies in fp16's
-    //      normal range whatever the norms are (tiny, huge or mixed), and the
-    //      hi/lo split of P keeps its ~22 bits.  Lloyd-Max: |v| is the stored
-    //      fp16 norm, ev its exponent (subnormals and zero as 2^-14).  Affine:
-    //      ev is the exponent of the token's largest |scale| or |bias| (clamped
-    //      to [-14, 14]); the value side scales (scale, bias) by 2^-ev exactly.
+    // ---- value magnitude of tokens g, g + 8: ev ~ log2 |v| and the factor
+    //      vm = |v| that stays with the weight.  The running maximum below is
+    //      taken over s + ev, so every weight p * |v| = 2^(s - max) |v| stays
+    //      below 2^(lazy slack) whatever the norms are (tiny, huge or mixed)
+    //      and the hi/lo split of P keeps its ~22 bits in fp16's normal range.
+    //      Lloyd-Max: |v| is the stored fp16 norm and ev its hardware log2
+    //      (2^-30 added, so a zero norm gives -30).  Affine: |v| = 2^ev with ev
+    //      the exponent of the token's largest |scale| or |bias| (clamped to
+    //      [-14, 14]); the value side scales (scale, bias) by 2^-ev exactly.
     float vm0, vm1, ev0, ev1;
     uint32_t vfac = 0u;  // affine: fp16 bits of 2^-ev of tokens g (low) and g + 8 (high)
     if constexpr (!AFF) {
@@ -865,8 +904,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       const uint32_t b0 = vn[g], b1 = vn[g + 8];
       vm0 = __half2float(__ushort_as_half((uint16_t)b0));
       vm1 = __half2float(__ushort_as_half((uint16_t)b1));
-      ev0 = (float)(max((int)((b0 >> 10) & 31u), 1) - 15);
-      ev1 = (float)(max((int)((b1 >> 10) & 31u), 1) - 15);
+      ev0 = ok0 ? fast_log2(vm0 + 0x1p-30f) : 0.f;  // zero norms give -30
+      ev1 = ok1 ? fast_log2(vm1 + 0x1p-30f) : 0.f;
     } else {
       const uint32_t* vmw = reinterpret_cast<const uint32_t*>(st + Geo::offVN) + (r0 + g) * Geo::NG;
       uint32_t f0 = 1u, f1 = 1u;  // largest fp16 exponent field among |scale|, |bias|
@@ -1086,8 +1125,19 @@ template <int D, int G, int KB, int VB, bool QJL, bool AFF>
 cudaError_t configure_shape(int* ctas_per_sm) {
   using Geo = DecodeGeom<D, G, KB, VB, QJL, AFF>;
   static KernelConfig cfg;  // one per shape
-  return configure_kernel(cfg, decode_kernel<D, G, KB, VB, QJL, AFF>, Geo::total, kDecThreads,
-                          ctas_per_sm);
+  auto kern = decode_kernel<D, G, KB, VB, QJL, AFF>;
+  // the dynamic shared memory must start at kDynSmemBase: no static shared
+  // memory, and the per-CTA reserved shared memory of that size
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  int dev = 0, reserved = -1;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  if (fa.sharedSizeBytes != 0 || reserved != (int)kDynSmemBase) return cudaErrorNotSupported;
+  return configure_kernel(cfg, kern, Geo::total, kDecThreads, ctas_per_sm);
 }
 
 // Launches decode_kernel for one compile-time shape (grid: plan.ctas CTAs).

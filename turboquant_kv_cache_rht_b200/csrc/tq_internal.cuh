@@ -19,6 +19,7 @@ __device__ __forceinline__ void pdl_trigger() {
 
 constexpr unsigned kFlagCapacity = 1u;  // mirrors TQ_FLAG_CAPACITY
 constexpr unsigned kFlagMaxCtx = 2u;    // mirrors TQ_FLAG_MAXCTX
+constexpr unsigned kFlagLayout = 4u;    // mirrors TQ_FLAG_LAYOUT
 
 // Codebooks and rotation signs, passed to every kernel by value (they live in
 // the kernel parameter bank; no device allocation is needed).

@@ -26,6 +26,7 @@ lib = C.CDLL(_LIB_PATH)
 TQ_OK, TQ_ERR_INVALID, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_CAPACITY, TQ_ERR_NOMEM = range(6)
 TQ_FLAG_CAPACITY = 1
 TQ_FLAG_MAXCTX = 2
+TQ_FLAG_LAYOUT = 4
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EXPORTS = ("tq_codebook_init", "tq_codebook_tables", "tq_quantize_append", "tq_quantize_cache",
            "tq_weights_quantize", "tq_lut_matmul_workspace_bytes", "tq_lut_matmul",
