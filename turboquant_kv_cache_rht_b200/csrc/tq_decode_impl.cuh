@@ -142,6 +142,13 @@ __device__ __forceinline__ uint32_t lds_table(uint32_t idx) {
   return v;
 }
 
+template <uint32_t OFF>
+__device__ __forceinline__ uint2 lds_table64(uint32_t idx) {
+  uint2 v;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(idx), "n"(OFF));
+  return v;
+}
+
 // (a, b) -> half2 of their fp16 roundings (hi) and of the remainders (lo).
 __device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -232,16 +239,27 @@ struct DecodeGeom {
   static constexpr int VCH = VB * D / 8;      // value bits per thread group
   static constexpr int VCW = (VCH + 31) / 32; // words of the aligned value chunk
   static constexpr int VNW = (VCH % 32 == 0) ? VCH / 32 : (VCH + 16 + 31) / 32;
-  static constexpr int LK = 1 << (2 * KB);    // key pair-table entries (4 bytes: an fp16 pair)
-  static constexpr int LV = 1 << (2 * VB);    // value pair-table entries (4 bytes each)
+  // 2-bit codes take quad tables: a byte of four codes -> four fp16 values (8
+  // bytes), one 64-bit lookup per two MMA registers; wider codes take pair
+  // tables (two codes -> an fp16 pair, 4 bytes).  The affine codec keeps pairs.
+  static constexpr bool QK = KB == 2 && !AFF;  // quad key table
+  static constexpr bool QV = VB == 2 && !AFF;  // quad value table
+  static constexpr int LK = QK ? 256 : 1 << (2 * KB);  // key table entries
+  static constexpr int LV = QV ? 256 : 1 << (2 * VB);  // value table entries
+  static constexpr int EKL = QK ? 3 : 2;               // log2 bytes of a key entry
+  static constexpr int EVL = QV ? 3 : 2;               // log2 bytes of a value entry
   // Each table is replicated so that lanes with different (lane mod copies)
   // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * 4.
   // 32 copies (a lane's own) keep every lookup free of bank conflicts; the
   // 4-bit tables of head_dim 256 keep 16 to leave room for the stages
-  static constexpr int RKL = (KB <= 3 || D <= 128) ? 5 : 4;  // log2 key copies
-  static constexpr int RVL = (VB <= 3 || D <= 128) ? 5 : 4;  // log2 value copies
-  static constexpr int KSH = 2 + RKL;          // byte shift of a key entry index
-  static constexpr int VSH = 2 + RVL;          // byte shift of a value entry index
+  // (64-bit lookups are served per half-warp, so 16 copies already keep the
+  // quad tables free of conflicts)
+  static constexpr int RKL = QK ? 4 : (KB <= 3 || D <= 128) ? 5 : 4;  // log2 key copies
+  static constexpr int RVL = QV ? 4 : (VB <= 3 || D <= 128) ? 5 : 4;  // log2 value copies
+  static constexpr int KSH = EKL + RKL;        // byte shift of a key entry index
+  static constexpr int VSH = EVL + RVL;        // byte shift of a value entry index
+  // value quads: y / z bytes per interleaved word (a byte holds two channels)
+  static constexpr int BPW = D / 32 < 4 ? D / 32 : 4;
   // affine codec: NG groups of 64 channels, one (scale, bias) word per group
   // and token; thread quarter qd reads channels [64 gg + 16 qd, + 16) of group gg
   static constexpr int NG = D / kAffineGroup;
@@ -264,8 +282,8 @@ struct DecodeGeom {
       (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
   // after the stage area
   static constexpr int offLK = stagesBytes;
-  static constexpr int offLV = offLK + (LK << RKL) * 4;
-  static constexpr int offQ = offLV + (LV << RVL) * 4;         // float [G][D] rotated query
+  static constexpr int offLV = offLK + (LK << RKL << EKL);
+  static constexpr int offQ = offLV + (LV << RVL << EVL);      // float [G][D] rotated query
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
   static constexpr int offRed = offUs + (AFF ? (G * NG * 4 + 15) / 16 * 16 : 0);  // float scratch
@@ -324,6 +342,17 @@ __device__ __forceinline__ void interleave_pairs(const uint32_t (&a)[VCW], const
       z[w] = b[w];
     }
   }
+}
+
+// Channel, within a thread group's D/8 value channels, of MMA row g (h = 0) or
+// g + 8 (h = 1) of m-block mb: consecutive channels 2mb, 2mb + 1 with pair
+// tables; with quad tables m-block mb reads byte `by` of the even (y) or odd
+// (z) interleaved word w, whose two codes are channels c and c + 2.
+template <bool QV, int BPW>
+__host__ __device__ constexpr int value_channel(int mb, int h) {
+  if (!QV) return 2 * mb + h;
+  const int w = mb / (2 * BPW), r = mb % (2 * BPW);
+  return 16 * w + 4 * (r % BPW) + 2 * h + (r < BPW ? 0 : 1);
 }
 
 // Byte offsets, into this lane's copy of the value pair table, of the pairs
@@ -422,19 +451,35 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   {
     // each entry is computed once and written to all its copies with 16-byte stores
     constexpr int RK = 1 << Geo::RKL, RV = 1 << Geo::RVL;
+    auto quad = [&](const float* c, float lam, int p) {  // byte of four 2-bit codes
+      return make_uint2(pack_half2(__float2half_rn(c[p & 3] * lam), __float2half_rn(c[(p >> 2) & 3] * lam)),
+                        pack_half2(__float2half_rn(c[(p >> 4) & 3] * lam), __float2half_rn(c[(p >> 6) & 3] * lam)));
+    };
     for (int p = tid; p < Geo::LK; p += kDecThreads) {
-      const uint32_t k = pack_half2(__float2half_rn(tb.k_cent[p & ((1 << KB) - 1)] * tb.k_lam),
-                                    __float2half_rn(tb.k_cent[p >> KB] * tb.k_lam));
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 4);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * ((RK << Geo::EKL) / 16);
+      if constexpr (Geo::QK) {
+        const uint2 k = quad(tb.k_cent, tb.k_lam, p);
 #pragma unroll
-      for (int c = 0; c < RK / 4; ++c) dst[c] = make_uint4(k, k, k, k);
+        for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(k.x, k.y, k.x, k.y);
+      } else {
+        const uint32_t k = pack_half2(__float2half_rn(tb.k_cent[p & ((1 << KB) - 1)] * tb.k_lam),
+                                      __float2half_rn(tb.k_cent[p >> KB] * tb.k_lam));
+#pragma unroll
+        for (int c = 0; c < RK / 4; ++c) dst[c] = make_uint4(k, k, k, k);
+      }
     }
     for (int p = tid; p < Geo::LV; p += kDecThreads) {
-      const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)] * tb.v_lam),
-                                    __float2half_rn(tb.v_cent[p >> VB] * tb.v_lam));
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * (RV / 4);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * ((RV << Geo::EVL) / 16);
+      if constexpr (Geo::QV) {
+        const uint2 v = quad(tb.v_cent, tb.v_lam, p);
 #pragma unroll
-      for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
+        for (int c = 0; c < RV / 2; ++c) dst[c] = make_uint4(v.x, v.y, v.x, v.y);
+      } else {
+        const uint32_t v = pack_half2(__float2half_rn(tb.v_cent[p & ((1 << VB) - 1)] * tb.v_lam),
+                                      __float2half_rn(tb.v_cent[p >> VB] * tb.v_lam));
+#pragma unroll
+        for (int c = 0; c < RV / 4; ++c) dst[c] = make_uint4(v, v, v, v);
+      }
     }
   }
 
@@ -687,8 +732,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][mb][e] = 0.f;
   }
-  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 2;
-  const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << 2;
+  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << Geo::EKL;
+  const uint32_t v_lane = (uint32_t)(lane & ((1 << Geo::RVL) - 1)) << Geo::EVL;
   const int src1 = 8 * qd + (g >> 1), src2 = src1 + 4;  // lanes holding P of tokens 2q(+8), 2q+1(+9)
 
   // value aggregation of the warp's previous slab, run at the top of its next
@@ -707,13 +752,29 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     interleave_pairs<VB, Geo::VCW>(pvc, pvd, y1, z1);
 #pragma unroll
     for (int mb = 0; mb < Geo::MBLK; ++mb) {
-      uint32_t e0, o0, e1, o1;
-      value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
-      value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
-      uint32_t a0 = lds_table<kDynSmemBase + Geo::offLV>(e0);
-      uint32_t a1 = lds_table<kDynSmemBase + Geo::offLV>(o0);
-      uint32_t a2 = lds_table<kDynSmemBase + Geo::offLV>(e1);
-      uint32_t a3 = lds_table<kDynSmemBase + Geo::offLV>(o1);
+      uint32_t a0, a1, a2, a3;
+      if constexpr (Geo::QV) {
+        // byte `by` of y (even channels) or z (odd channels) of word w holds
+        // channels c and c + 2 of tokens (a, b): rows g and g + 8 of m-block mb
+        constexpr int BPW = Geo::BPW;
+        const int w = mb / (2 * BPW), r = mb % (2 * BPW), by = r % BPW;
+        const uint32_t* s0 = r < BPW ? y0 : z0;
+        const uint32_t* s1 = r < BPW ? y1 : z1;
+        const uint2 q0 = lds_table64<kDynSmemBase + Geo::offLV>(bits_at(s0[w], 8 * by, 8, Geo::VSH) | v_lane);
+        const uint2 q1 = lds_table64<kDynSmemBase + Geo::offLV>(bits_at(s1[w], 8 * by, 8, Geo::VSH) | v_lane);
+        a0 = q0.x;
+        a1 = q0.y;
+        a2 = q1.x;
+        a3 = q1.y;
+      } else {
+        uint32_t e0, o0, e1, o1;
+        value_pairs<VB, Geo::VCW, Geo::VSH>(y0, z0, mb, v_lane, e0, o0);
+        value_pairs<VB, Geo::VCW, Geo::VSH>(y1, z1, mb, v_lane, e1, o1);
+        a0 = lds_table<kDynSmemBase + Geo::offLV>(e0);
+        a1 = lds_table<kDynSmemBase + Geo::offLV>(o0);
+        a2 = lds_table<kDynSmemBase + Geo::offLV>(e1);
+        a3 = lds_table<kDynSmemBase + Geo::offLV>(o1);
+      }
       if constexpr (AFF) {  // integer levels -> scale * level + bias of each token
         a0 = hfma2_bits(psab, a0, pbab);
         a1 = hfma2_bits(psab, a1, pbab);
@@ -783,10 +844,20 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
         for (int kb = 0; kb < Geo::KBLK; ++kb) {
           const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
-          const uint32_t a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
-          const uint32_t a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
-          const uint32_t a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
-          const uint32_t a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+          uint32_t a0, a1, a2, a3;
+          if constexpr (Geo::QK) {  // the byte of channels c0 .. c0+3: one quad per token
+            const uint2 p = lds_table64<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 8, Geo::KSH) | k_lane);
+            const uint2 q = lds_table64<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 8, Geo::KSH) | k_lane);
+            a0 = p.x;
+            a1 = q.x;
+            a2 = p.y;
+            a3 = q.y;
+          } else {
+            a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+            a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+            a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+            a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+          }
 #pragma unroll
           for (int j = 0; j < NT; ++j) mma16816(sacc[kb & 1][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
         }
@@ -1010,8 +1081,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       float* o = ow + (warp * G + head) * D + g * (D / 8);
 #pragma unroll
       for (int mb = 0; mb < Geo::MBLK; ++mb) {
-        o[2 * mb] = acc[j][mb][0] + acc[j][mb][1];
-        o[2 * mb + 1] = acc[j][mb][2] + acc[j][mb][3];
+        o[value_channel<Geo::QV, Geo::BPW>(mb, 0)] = acc[j][mb][0] + acc[j][mb][1];
+        o[value_channel<Geo::QV, Geo::BPW>(mb, 1)] = acc[j][mb][2] + acc[j][mb][3];
       }
     }
   }
