@@ -113,7 +113,7 @@ template <int E>
 __device__ __forceinline__ void flip_signs(float (&u)[E], const uint32_t* mask, int g) {
   const uint32_t bits = mask[(g * E) >> 5] >> ((g * E) & 31);
 #pragma unroll
-  for (int e = 0; e < E; ++e) u[e] = __uint_as_float(__float_as_uint(u[e]) ^ (((bits >> e) & 1u) << 31));
+  for (int e = 0; e < E; ++e) u[e] = __uint_as_float(__float_as_uint(u[e]) ^ ((bits << (31 - e)) & 0x80000000u));
 }
 
 // Stores a packed row whose lanes each hold `width` (< 32) consecutive bits at

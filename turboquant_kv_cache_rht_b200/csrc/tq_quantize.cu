@@ -62,16 +62,21 @@ __device__ __forceinline__ void encode_vector(int bits, float (&u)[E], const Tab
 }
 constexpr int kAppendThreads = 32 * kAppendWarps;
 
-// Grid: (2 * blocks_per_kind, batch).  Blocks [0, blocks_per_kind) encode keys,
-// the rest values, so a block's code width is uniform.  A group of D / E lanes
+// Grid: (kinds * blocks_per_kind, batch).  Blocks encode kind `first_kind`
+// (0 keys, 1 values), the next blocks_per_kind blocks the other kind when
+// kinds is 2, so a block's code width is uniform.  A group of D / E lanes
 // encodes one vector: E = 32 packs 32 * 32 / D vectors into a warp (throughput:
 // bulk appends); E = D / 32 gives each vector its own warp and keeps the
 // unrolled code short (latency: a few tokens per row, as in a decode step).
+// `publish`: this grid's last block of a row sets the row's new length (a
+// bulk append runs keys and values as two grids, so that each grid executes
+// one code width and its unrolled code stays in the instruction cache; the
+// second grid publishes).
 template <int D, typename T, int E, bool AFF>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_append_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                            const T* __restrict__ kin, const T* __restrict__ vin, int n_new,
-                           int blocks_per_kind) {
+                           int blocks_per_kind, int first_kind, int publish) {
   constexpr int GL = D / E;                     // lanes per vector
   constexpr int VPB = kAppendThreads / GL;      // vectors per block
   __shared__ float s_kcent[16];
@@ -80,8 +85,9 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int tid = threadIdx.x, lane = tid & 31, g = lane & (GL - 1);
   if (tid < 16) s_kcent[tid] = tb.k_cent[tid];
   const int b = blockIdx.y;
-  const bool is_v = (int)blockIdx.x >= blocks_per_kind;
-  const long r = (long)(blockIdx.x - (is_v ? blocks_per_kind : 0)) * VPB + tid / GL;
+  const int kind_block = (int)blockIdx.x / blocks_per_kind;
+  const bool is_v = first_kind + kind_block == 1;
+  const long r = (long)((int)blockIdx.x - kind_block * blocks_per_kind) * VPB + tid / GL;
   const long per_kind = (long)cv.kv_heads * n_new;
   const bool valid = r < per_kind;
   const int h = valid ? (int)(r / n_new) : 0, j = valid ? (int)(r % n_new) : 0;
@@ -121,13 +127,15 @@ __global__ void __launch_bounds__(kAppendThreads)
 
   // The last block of this batch row to finish publishes the new length.  Every
   // block read seq_lens[b] before taking its ticket, so none can see the update.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const int ticket = atomicAdd(&cv.append_sync[b], 1);
-    if (ticket == (int)gridDim.x - 1) {
-      if (fits) cv.seq_lens[b] = base + n_new;
-      cv.append_sync[b] = 0;
+  if (publish) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      const int ticket = atomicAdd(&cv.append_sync[b], 1);
+      if (ticket == (int)gridDim.x - 1) {
+        if (fits) cv.seq_lens[b] = base + n_new;
+        cv.append_sync[b] = 0;
+      }
     }
   }
   if constexpr (E == 32) pdl_trigger();
@@ -144,7 +152,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     quantize_convert_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                             const T* __restrict__ kin, const T* __restrict__ vin, long stride_b,
                             long stride_h, long stride_t, const int32_t* __restrict__ lengths,
-                            int max_len, int blocks_per_kind, int heads_inner) {
+                            int max_len, int blocks_per_kind, int heads_inner, int first_kind) {
   constexpr int GL = D / E;
   constexpr int VPB = kAppendThreads / GL;
   __shared__ float s_kcent[16];
@@ -153,8 +161,9 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int tid = threadIdx.x, lane = tid & 31, g = lane & (GL - 1);
   if (tid < 16) s_kcent[tid] = tb.k_cent[tid];
   const int b = blockIdx.y, H = cv.kv_heads;
-  const bool is_v = (int)blockIdx.x >= blocks_per_kind;
-  const long r = (long)(blockIdx.x - (is_v ? blocks_per_kind : 0)) * VPB + tid / GL;
+  const int kind_block = (int)blockIdx.x / blocks_per_kind;
+  const bool is_v = first_kind + kind_block == 1;
+  const long r = (long)((int)blockIdx.x - kind_block * blocks_per_kind) * VPB + tid / GL;
   const bool in_grid = r < (long)H * max_len;
   const int h = !in_grid ? 0 : heads_inner ? (int)(r % H) : (int)(r / max_len);
   const int t = !in_grid ? 0 : heads_inner ? (int)(r / H) : (int)(r % max_len);
@@ -200,6 +209,10 @@ __global__ void __launch_bounds__(kAppendThreads)
 // latency rules; larger ones take the 32-channels-per-lane layout.
 constexpr long kLatencyVectors = 4096;
 
+// One grid over both kinds (small appends: one launch, latency) or, for the
+// bulk layout, a grid of keys followed by a grid of values (each grid runs one
+// code width, which keeps its unrolled encoder resident in the instruction
+// cache); the grid that runs last publishes the lengths.
 template <int D, typename T, int E, bool AFF>
 cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                           int n_new, cudaStream_t stream) {
@@ -208,7 +221,6 @@ cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, 
   const long blocks_per_kind = std::max<long>(1, (per_kind + VPB - 1) / VPB);
   if (2 * blocks_per_kind > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * blocks_per_kind), (unsigned)cv.batch);
   cfg.blockDim = dim3(kAppendThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -216,9 +228,18 @@ cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_append_kernel<D, T, E, AFF>, tb, cv,
-                            static_cast<const T*>(k), static_cast<const T*>(v), n_new,
-                            (int)blocks_per_kind);
+  auto kern = quantize_append_kernel<D, T, E, AFF>;
+  const T* kp = static_cast<const T*>(k);
+  const T* vp = static_cast<const T*>(v);
+  if constexpr (E < 32) {
+    cfg.gridDim = dim3((unsigned)(2 * blocks_per_kind), (unsigned)cv.batch);
+    return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 1);
+  } else {
+    cfg.gridDim = dim3((unsigned)blocks_per_kind, (unsigned)cv.batch);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 0);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 1, 1);
+  }
 }
 
 template <int D, typename T>
@@ -243,7 +264,6 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
   const long blocks_per_kind = std::max<long>(1, (per_kind + VPB - 1) / VPB);
   if (kinds * blocks_per_kind > 0x7fffffffL || cv.batch > 65535) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(kinds * blocks_per_kind), (unsigned)cv.batch);
   cfg.blockDim = dim3(kAppendThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -251,9 +271,19 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_convert_kernel<D, T, E, AFF>, tb, cv,
-                            static_cast<const T*>(k), static_cast<const T*>(v), sb, sh, st,
-                            lengths, max_len, (int)blocks_per_kind, sh < st ? 1 : 0);
+  auto kern = quantize_convert_kernel<D, T, E, AFF>;
+  const T* kp = static_cast<const T*>(k);
+  const T* vp = static_cast<const T*>(v);
+  const int heads_inner = sh < st ? 1 : 0;
+  // the bulk layout runs keys and values as two grids (one code width each,
+  // as for the append)
+  const bool split = E == 32 && kinds == 2;
+  cfg.gridDim = dim3((unsigned)((split ? 1 : kinds) * blocks_per_kind), (unsigned)cv.batch);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
+                                     (int)blocks_per_kind, heads_inner, 0);
+  if (e != cudaSuccess || !split) return e;
+  return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
+                            (int)blocks_per_kind, heads_inner, 1);
 }
 
 template <int D, typename T>
