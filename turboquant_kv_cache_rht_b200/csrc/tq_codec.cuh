@@ -116,19 +116,26 @@ __device__ __forceinline__ void flip_signs(float (&u)[E], const uint32_t* mask, 
   for (int e = 0; e < E; ++e) u[e] = __uint_as_float(__float_as_uint(u[e]) ^ ((bits << (31 - e)) & 0x80000000u));
 }
 
-// Stores a packed row whose lanes each hold `width` (< 32) consecutive bits at
-// stream bit lane * width: the warp ORs the chunks into a shared word buffer
-// and writes the `words` words (one vector per warp; every lane calls).
-__device__ __forceinline__ void pack_store_shared(uint32_t* buf, int words, uint32_t chunk,
-                                                  int width, int lane, bool store, uint32_t* dst) {
-  if (lane < words) buf[lane] = 0u;
-  __syncwarp();
-  const int off = lane * width, w = off >> 5, sh = off & 31;
-  atomicOr(&buf[w], chunk << sh);
-  if (sh + width > 32) atomicOr(&buf[w + 1], chunk >> (32 - sh));
-  __syncwarp();
-  if (store && lane < words) dst[lane] = buf[lane];
-  __syncwarp();
+// Stores a packed row whose GL lanes (g = 0 .. GL-1 of the vector's group) each
+// hold LB (< 32) consecutive bits at stream bit g * LB: lane g < W assembles
+// word g of the row from the chunks of the lanes it spans (shuffles within
+// the group, no shared memory) and stores it.  Every lane of the group calls.
+template <int GL, int LB>
+__device__ __forceinline__ void pack_store_shuffle(uint32_t chunk, int g, int lane, bool store,
+                                                   uint32_t* dst) {
+  static_assert(LB < 32 && (LB * GL) % 32 == 0, "sub-word chunks that fill whole words");
+  constexpr int W = LB * GL / 32;          // words of the row
+  constexpr int NS = (31 + LB - 1) / LB + 1;  // lanes one word can span
+  const int base = lane - g, first = (32 * g) / LB, off = 32 * g - first * LB;
+  uint32_t word = 0u;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    const int src = first + i;
+    const uint32_t c = __shfl_sync(kFull, chunk, base + (src < GL ? src : GL - 1), 32);
+    const int pos = i * LB - off;  // where bit 0 of lane src's chunk lands in the word
+    if (src < GL && pos < 32 && pos > -LB) word |= pos >= 0 ? (c << pos) : (c >> -pos);
+  }
+  if (store && g < W) dst[g] = word;
 }
 
 // #{q : p[q] < key} for the P = 2^(B-1) - 1 positive boundaries p (ascending),
@@ -168,8 +175,7 @@ __device__ __forceinline__ int bucket(float z, const float (&p)[8]) {
 // the packed row at stream bit g * LB.
 template <int D, int E, int B>
 __device__ __forceinline__ void store_codes(const uint32_t (&words)[(B * E + 31) / 32], int g,
-                                            int lane, bool store, uint8_t* codes_row,
-                                            uint32_t* pack) {
+                                            int lane, bool store, uint8_t* codes_row) {
   constexpr int LB = B * E;
   if constexpr (LB % 32 == 0) {
     if (store) {
@@ -178,8 +184,7 @@ __device__ __forceinline__ void store_codes(const uint32_t (&words)[(B * E + 31)
       for (int w = 0; w < LB / 32; ++w) dst[w] = words[w];
     }
   } else {
-    pack_store_shared(pack, B * D / 32, words[0], LB, lane, store,
-                      reinterpret_cast<uint32_t*>(codes_row));
+    pack_store_shuffle<D / E, LB>(words[0], g, lane, store, reinterpret_cast<uint32_t*>(codes_row));
   }
 }
 
@@ -188,7 +193,7 @@ __device__ __forceinline__ void store_codes(const uint32_t (&words)[(B * E + 31)
 template <int D, int E>
 __device__ __forceinline__ void store_sketch(float (&u)[E], const Tables& tb, float rdiv, int g,
                                              int lane, bool store, uint8_t* signs_row,
-                                             uint16_t* rnorm, uint32_t* pack) {
+                                             uint16_t* rnorm) {
   constexpr int GL = D / E;
   float sq[E];
 #pragma unroll
@@ -202,7 +207,7 @@ __device__ __forceinline__ void store_sketch(float (&u)[E], const Tables& tb, fl
   if constexpr (E % 32 == 0) {
     if (store) reinterpret_cast<uint32_t*>(signs_row)[g] = sbits;
   } else {
-    pack_store_shared(pack, D / 32, sbits, E, lane, store, reinterpret_cast<uint32_t*>(signs_row));
+    pack_store_shuffle<D / E, E>(sbits, g, lane, store, reinterpret_cast<uint32_t*>(signs_row));
   }
   if (store && g == 0) *rnorm = __half_as_ushort(__float2half_rn(rho));
 }
@@ -210,14 +215,13 @@ __device__ __forceinline__ void store_sketch(float (&u)[E], const Tables& tb, fl
 // Encodes the vector whose E-channel slice this lane holds in u (fp32) and
 // stores codes, norm and, for QJL keys, the sketch.  g is the lane's index in
 // its group of D / E lanes; `store` is false for lanes of a group past the
-// end (they still take part in the group's shuffles).  `pack` is the warp's
-// word buffer, used when a lane's bits do not fill whole words (E < 32, one
-// vector per warp).
+// end (they still take part in the group's shuffles).  When a lane's bits do
+// not fill whole words, the group assembles the words by shuffles.
 template <int D, int E, int B>
 __device__ __forceinline__ void encode_store(float (&u)[E], const Tables& tb, bool is_v, int g,
                                              int lane, bool store, uint8_t* codes_row,
                                              uint16_t* norm, uint8_t* signs_row, uint16_t* rnorm,
-                                             const float* s_kcent, uint32_t* pack) {
+                                             const float* s_kcent) {
   constexpr int GL = D / E;
   constexpr int H = 1 << (B - 1);
   constexpr int LB = B * E;  // code bits per lane
@@ -253,11 +257,11 @@ __device__ __forceinline__ void encode_store(float (&u)[E], const Tables& tb, bo
     // QJL keys: the residual r = u - fp16(n) * c[code] replaces u
     if (qjl) u[e] = __fsub_rn(u[e], __fmul_rn(n16f, s_kcent[c]));
   }
-  store_codes<D, E, B>(words, g, lane, store, codes_row, pack);
+  store_codes<D, E, B>(words, g, lane, store, codes_row);
   if (store && g == 0) *norm = __half_as_ushort(n16);
 
   // 6.-8. QJL sketch of keys: rho = ||r|| / sqrt(d); sign bits of H (s2 * r)
-  if (qjl) store_sketch<D, E>(u, tb, __fsqrt_rn((float)D), g, lane, store, signs_row, rnorm, pack);
+  if (qjl) store_sketch<D, E>(u, tb, __fsqrt_rn((float)D), g, lane, store, signs_row, rnorm);
 }
 
 // The affine group-64 comparison codec ("mlx-turboquant" README, "Quantize
@@ -273,8 +277,7 @@ template <int D, int E, int B>
 __device__ __forceinline__ void encode_affine_store(float (&u)[E], const Tables& tb, bool is_v,
                                                     int g, int lane, bool store,
                                                     uint8_t* codes_row, uint32_t* meta,
-                                                    uint8_t* signs_row, uint16_t* rnorm,
-                                                    uint32_t* pack) {
+                                                    uint8_t* signs_row, uint16_t* rnorm) {
   constexpr int GL = D / E;
   constexpr int LB = B * E;
   constexpr int GG = kAffineGroup / E;  // lanes per channel group (2 .. 32)
@@ -319,10 +322,10 @@ __device__ __forceinline__ void encode_affine_store(float (&u)[E], const Tables&
     if (s + B > 32) words[w + 1] |= (uint32_t)c >> (32 - s);
     if (qjl) u[e] = __fsub_rn(u[e], __fadd_rn(__fmul_rn(sf, (float)c), bf));
   }
-  store_codes<D, E, B>(words, g, lane, store, codes_row, pack);
+  store_codes<D, E, B>(words, g, lane, store, codes_row);
   if (store && g % GG == 0)
     meta[g / GG] = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(b16) << 16);
-  if (qjl) store_sketch<D, E>(u, tb, 1.0f, g, lane, store, signs_row, rnorm, pack);
+  if (qjl) store_sketch<D, E>(u, tb, 1.0f, g, lane, store, signs_row, rnorm);
 }
 
 }  // namespace codec

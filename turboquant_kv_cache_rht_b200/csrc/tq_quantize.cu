@@ -9,12 +9,15 @@
 // instantiated for the affine group-64 comparison codec (rotated keys, fp16
 // scale and bias per group of 64 channels: encode_affine_store).
 //
-// A group of d/32 adjacent lanes encodes one vector, each lane holding 32
-// consecutive channels, so a warp encodes 32*32/d vectors at once.  Five of
-// the transform's butterfly stages and five levels of the norm's pairwise tree
-// run inside a lane; the rest are shuffles within the group.  A lane's 32
-// codes fill whole 32-bit words of the packed row, so packing needs no
-// cross-lane traffic.
+// Bulk layout: a group of d/32 adjacent lanes encodes one vector, each lane
+// holding 32 consecutive channels, so a warp encodes 32*32/d vectors at once.
+// Five of the transform's butterfly stages and five levels of the norm's
+// pairwise tree run inside a lane; the rest are shuffles within the group.  A
+// lane's 32 codes fill whole 32-bit words of the packed row, so packing needs
+// no cross-lane traffic.  (Eight channels per lane, measured as well, runs 1.7x
+// the instructions at a higher issue rate and is 30% slower.)  Small appends
+// give each vector a warp (d/32 channels per lane); their lanes' codes are
+// assembled into words by shuffles.
 //
 // Every floating-point step is a single correctly rounded fp32 operation in
 // one fixed order (__fadd_rn / __fsub_rn / __fmul_rn / __fsqrt_rn /
@@ -35,6 +38,8 @@ namespace {
 using namespace codec;
 
 constexpr int kAppendWarps = 8;
+// Channels per lane of the bulk layout (appends of many vectors, conversion).
+constexpr int kBulkE = 32;
 
 // The codec of one vector at its code width: Lloyd-Max (norm, codes, sketch)
 // or the affine group-64 comparison codec (scale/bias pairs in `norm`).
@@ -42,22 +47,22 @@ template <int D, int E, bool AFF>
 __device__ __forceinline__ void encode_vector(int bits, float (&u)[E], const Tables& tb, bool is_v,
                                               int g, int lane, bool valid, uint8_t* codes,
                                               uint16_t* norm, uint8_t* signs, uint16_t* rnorm,
-                                              const float* s_kcent, uint32_t* pack) {
+                                              const float* s_kcent) {
   if constexpr (AFF) {
     uint32_t* meta = reinterpret_cast<uint32_t*>(norm);
     if (bits == 2)
-      encode_affine_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+      encode_affine_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm);
     else if (bits == 3)
-      encode_affine_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+      encode_affine_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm);
     else
-      encode_affine_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm, pack);
+      encode_affine_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm);
   } else {
     if (bits == 2)
-      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+      encode_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
     else if (bits == 3)
-      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+      encode_store<D, E, 3>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
     else
-      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent, pack);
+      encode_store<D, E, 4>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
   }
 }
 constexpr int kAppendThreads = 32 * kAppendWarps;
@@ -72,7 +77,7 @@ constexpr int kAppendThreads = 32 * kAppendWarps;
 // bulk append runs keys and values as two grids, so that each grid executes
 // one code width and its unrolled code stays in the instruction cache; the
 // second grid publishes).
-template <int D, typename T, int E, bool AFF>
+template <int D, typename T, int E, bool AFF, bool BULK>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_append_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                            const T* __restrict__ kin, const T* __restrict__ vin, int n_new,
@@ -80,7 +85,6 @@ __global__ void __launch_bounds__(kAppendThreads)
   constexpr int GL = D / E;                     // lanes per vector
   constexpr int VPB = kAppendThreads / GL;      // vectors per block
   __shared__ float s_kcent[16];
-  __shared__ uint32_t s_pack[kAppendWarps][E < 32 ? D / 8 + 1 : 1];
 
   const int tid = threadIdx.x, lane = tid & 31, g = lane & (GL - 1);
   if (tid < 16) s_kcent[tid] = tb.k_cent[tid];
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(kAppendThreads)
   // next kernel launch now, so that its set-up overlaps this one (it still waits
   // for this grid's completion before reading anything).  A bulk append keeps
   // the trigger at its end, so that waiting CTAs do not take its blocks' slots.
-  if constexpr (E < 32) pdl_trigger();
+  if constexpr (!BULK) pdl_trigger();
   const int base = cv.seq_lens[b];
   const bool fits = base >= 0 && base <= cv.capacity - n_new;
   if (!fits && tid == 0 && blockIdx.x == 0) atomicOr(cv.status, (int)kFlagCapacity);
@@ -120,9 +124,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
-    uint32_t* pack = s_pack[tid >> 5];
-    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent,
-                             pack);
+    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
   }
 
   // The last block of this batch row to finish publishes the new length.  Every
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kAppendThreads)
       }
     }
   }
-  if constexpr (E == 32) pdl_trigger();
+  if constexpr (BULK) pdl_trigger();
 }
 
 // Conversion of a dense cache.  Grid: (kinds * blocks_per_kind, batch) as for
@@ -156,7 +158,6 @@ __global__ void __launch_bounds__(kAppendThreads)
   constexpr int GL = D / E;
   constexpr int VPB = kAppendThreads / GL;
   __shared__ float s_kcent[16];
-  __shared__ uint32_t s_pack[kAppendWarps][E < 32 ? D / 8 + 1 : 1];
 
   const int tid = threadIdx.x, lane = tid & 31, g = lane & (GL - 1);
   if (tid < 16) s_kcent[tid] = tb.k_cent[tid];
@@ -197,9 +198,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
-    uint32_t* pack = s_pack[tid >> 5];
-    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent,
-                             pack);
+    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
   }
   pdl_trigger();
 }
@@ -213,7 +212,7 @@ constexpr long kLatencyVectors = 4096;
 // bulk layout, a grid of keys followed by a grid of values (each grid runs one
 // code width, which keeps its unrolled encoder resident in the instruction
 // cache); the grid that runs last publishes the lengths.
-template <int D, typename T, int E, bool AFF>
+template <int D, typename T, int E, bool AFF, bool BULK>
 cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, const void* v,
                           int n_new, cudaStream_t stream) {
   constexpr int VPB = kAppendThreads / (D / E);
@@ -228,10 +227,10 @@ cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  auto kern = quantize_append_kernel<D, T, E, AFF>;
+  auto kern = quantize_append_kernel<D, T, E, AFF, BULK>;
   const T* kp = static_cast<const T*>(k);
   const T* vp = static_cast<const T*>(v);
-  if constexpr (E < 32) {
+  if constexpr (!BULK) {
     cfg.gridDim = dim3((unsigned)(2 * blocks_per_kind), (unsigned)cv.batch);
     return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 1);
   } else {
@@ -247,17 +246,17 @@ cudaError_t launch_typed(const Tables& tb, const CacheView& cv, const void* k, c
                          int n_new, cudaStream_t stream) {
   const long vectors = 2L * cv.batch * cv.kv_heads * n_new;
   if (tb.affine) {
-    if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, true>(tb, cv, k, v, n_new, stream);
-    return launch_layout<D, T, 32, true>(tb, cv, k, v, n_new, stream);
+    if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, true, false>(tb, cv, k, v, n_new, stream);
+    return launch_layout<D, T, kBulkE, true, true>(tb, cv, k, v, n_new, stream);
   }
-  if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, false>(tb, cv, k, v, n_new, stream);
-  return launch_layout<D, T, 32, false>(tb, cv, k, v, n_new, stream);
+  if (vectors <= kLatencyVectors) return launch_layout<D, T, D / 32, false, false>(tb, cv, k, v, n_new, stream);
+  return launch_layout<D, T, kBulkE, false, true>(tb, cv, k, v, n_new, stream);
 }
 
 template <int D, typename T, int E, bool AFF>
 cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const void* k,
                                   const void* v, long sb, long sh, long st,
-                                  const int32_t* lengths, int max_len, int kinds,
+                                  const int32_t* lengths, int max_len, int kinds, bool small,
                                   cudaStream_t stream) {
   constexpr int VPB = kAppendThreads / (D / E);
   const long per_kind = (long)cv.kv_heads * max_len;
@@ -277,7 +276,7 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
   const int heads_inner = sh < st ? 1 : 0;
   // the bulk layout runs keys and values as two grids (one code width each,
   // as for the append)
-  const bool split = E == 32 && kinds == 2;
+  const bool split = !small && kinds == 2;
   cfg.gridDim = dim3((unsigned)((split ? 1 : kinds) * blocks_per_kind), (unsigned)cv.batch);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
                                      (int)blocks_per_kind, heads_inner, 0);
@@ -294,13 +293,13 @@ cudaError_t launch_convert_typed(const Tables& tb, const CacheView& cv, const vo
   const bool small = vectors <= kLatencyVectors;
   if (tb.affine)
     return small ? launch_convert_layout<D, T, D / 32, true>(tb, cv, k, v, sb, sh, st, lengths,
-                                                             max_len, kinds, stream)
-                 : launch_convert_layout<D, T, 32, true>(tb, cv, k, v, sb, sh, st, lengths, max_len,
-                                                         kinds, stream);
+                                                             max_len, kinds, true, stream)
+                 : launch_convert_layout<D, T, kBulkE, true>(tb, cv, k, v, sb, sh, st, lengths, max_len,
+                                                             kinds, false, stream);
   return small ? launch_convert_layout<D, T, D / 32, false>(tb, cv, k, v, sb, sh, st, lengths,
-                                                            max_len, kinds, stream)
-               : launch_convert_layout<D, T, 32, false>(tb, cv, k, v, sb, sh, st, lengths, max_len,
-                                                        kinds, stream);
+                                                            max_len, kinds, true, stream)
+               : launch_convert_layout<D, T, kBulkE, false>(tb, cv, k, v, sb, sh, st, lengths, max_len,
+                                                            kinds, false, stream);
 }
 
 template <int D>
