@@ -57,11 +57,11 @@ DECODE_SOURCES = ("tq_internal.cuh", "tq_decode_impl.cuh", "tq_decode.cu", "tq_d
                   "tq_decode_d256.cu", "tq_decode_affine_d64.cu", "tq_decode_affine_d128.cu",
                   "tq_decode_affine_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31754240, "35507a175a67dd52"),
-    "qjl": (566914304, "35507a175a67dd52"),
-    "long": (353341952, "35507a175a67dd52"),
-    "serving": (1102758656, "35507a175a67dd52"),
-    "affine": (38808064, "35507a175a67dd52"),
+    "gqa": (31446528, "beac15425fddc3fa"),
+    "qjl": (566852096, "beac15425fddc3fa"),
+    "long": (353267200, "beac15425fddc3fa"),
+    "serving": (1102322176, "beac15425fddc3fa"),
+    "affine": (38483456, "beac15425fddc3fa"),
 }
 
 
@@ -87,6 +87,23 @@ def decode_traffic(workload: str):
     if entry is None or entry[1] != decode_sources_digest():
         return None
     return entry[0]
+
+
+# Issue utilisation of the decode kernel per workload, from the ncu --set full
+# capture summarised in profiles/decode_kernel_<workload>.md: issue-active %
+# of active cycles, warp instructions per (token, KV head), warps active %.
+# Keyed, like the traffic, to the digest of the decode sources it describes.
+DECODE_PROFILE: dict[str, tuple[dict, str]] = {
+    "gqa": ({"issue_active_pct": 42.3, "warp_inst_per_token_head": 34.19, "warps_active_pct": 17.5}, "beac15425fddc3fa"),
+    "long": ({"issue_active_pct": 49.3, "warp_inst_per_token_head": 45.72, "warps_active_pct": 12.1}, "beac15425fddc3fa"),
+}
+
+
+def decode_profile(workload: str):
+    entry = DECODE_PROFILE.get(workload)
+    if entry is None or entry[1] != decode_sources_digest():
+        return None
+    return dict(entry[0], source=f"profiles/decode_kernel_{workload}.md")
 
 
 def peaks():
@@ -402,7 +419,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "roofline": {"bound": "hbm", "kernel": "tq_decode_attention (decode + combine launches)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(hbm_frac, 4), "traffic": decode_traffic(w.name),
-                     "algorithmic_bytes_per_launch": dec_bytes},
+                     "algorithmic_bytes_per_launch": dec_bytes,
+                     "issue": decode_profile(w.name)},
         "e2e": e2e,
         "gpu_launches": 3 * K,
         "clocks": clk.summary(),
