@@ -96,6 +96,8 @@ def decode_traffic(workload: str):
 DECODE_PROFILE: dict[str, tuple[dict, str]] = {
     "gqa": ({"issue_active_pct": 42.3, "warp_inst_per_token_head": 34.19, "warps_active_pct": 17.5}, "beac15425fddc3fa"),
     "long": ({"issue_active_pct": 49.3, "warp_inst_per_token_head": 45.72, "warps_active_pct": 12.1}, "beac15425fddc3fa"),
+    "qjl": ({"issue_active_pct": 59.4, "warp_inst_per_token_head": 34.33, "warps_active_pct": 17.2}, "beac15425fddc3fa"),
+    "serving": ({"issue_active_pct": 63.4, "warp_inst_per_token_head": 25.23, "warps_active_pct": 17.1}, "beac15425fddc3fa"),
 }
 
 
