@@ -256,8 +256,12 @@ struct DecodeGeom {
   // quad tables free of conflicts)
   static constexpr int RKL = QK ? 4 : (KB <= 3 || D <= 128) ? 5 : 4;  // log2 key copies
   static constexpr int RVL = QV ? 4 : (VB <= 3 || D <= 128) ? 5 : 4;  // log2 value copies
-  static constexpr int KSH = EKL + RKL;        // byte shift of a key entry index
-  static constexpr int VSH = EVL + RVL;        // byte shift of a value entry index
+  // When both tables are quads their 128-byte entries are interleaved, key
+  // entry e at byte 256 e and value entry e at 256 e + 128: an index is then
+  // the code byte above the lane's copy offset, which one byte permute forms.
+  static constexpr bool IQ = QK && QV;
+  static constexpr int KSH = IQ ? 8 : EKL + RKL;  // byte shift of a key entry index
+  static constexpr int VSH = IQ ? 8 : EVL + RVL;  // byte shift of a value entry index
   // value quads: y / z bytes per interleaved word (a byte holds two channels)
   static constexpr int BPW = D / 32 < 4 ? D / 32 : 4;
   // affine codec: NG groups of 64 channels, one (scale, bias) word per group
@@ -282,8 +286,8 @@ struct DecodeGeom {
       (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
   // after the stage area
   static constexpr int offLK = stagesBytes;
-  static constexpr int offLV = offLK + (LK << RKL << EKL);
-  static constexpr int offQ = offLV + (LV << RVL << EVL);      // float [G][D] rotated query
+  static constexpr int offLV = IQ ? offLK + 128 : offLK + (LK << KSH);
+  static constexpr int offQ = IQ ? offLK + (LK << 8) : offLV + (LV << VSH);  // float [G][D] rotated query
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
   static constexpr int offRed = offUs + (AFF ? (G * NG * 4 + 15) / 16 * 16 : 0);  // float scratch
@@ -321,6 +325,18 @@ __device__ __forceinline__ void load_value_chunk(const uint32_t* row, int g, uin
 __device__ __forceinline__ uint32_t bits_at(uint32_t x, int pos, int width, int scale) {
   const uint32_t mask = ((1u << width) - 1u) << scale;
   return pos >= scale ? (x >> (pos - scale)) & mask : (x << (scale - pos)) & mask;
+}
+
+// Index of the quad-table entry of byte `by` of x for a lane whose copy offset
+// is lane_off (< 256): with the interleaved layout (entry shift 8) the byte
+// permute places the code byte above the offset in one instruction.
+template <bool IQ, int SH>
+__device__ __forceinline__ uint32_t quad_index(uint32_t x, int by, uint32_t lane_off) {
+  if constexpr (IQ) {
+    return __byte_perm(x, lane_off, 0x5504u | ((uint32_t)by << 4));
+  } else {
+    return bits_at(x, 8 * by, 8, SH) | lane_off;
+  }
 }
 
 // Interleaves the value chunks of two tokens a, b so that each 2*VB-bit field
@@ -456,7 +472,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
                         pack_half2(__float2half_rn(c[(p >> 4) & 3] * lam), __float2half_rn(c[(p >> 6) & 3] * lam)));
     };
     for (int p = tid; p < Geo::LK; p += kDecThreads) {
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * ((RK << Geo::EKL) / 16);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK + (p << Geo::KSH));
       if constexpr (Geo::QK) {
         const uint2 k = quad(tb.k_cent, tb.k_lam, p);
 #pragma unroll
@@ -469,7 +485,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
       }
     }
     for (int p = tid; p < Geo::LV; p += kDecThreads) {
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV) + p * ((RV << Geo::EVL) / 16);
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLV + (p << Geo::VSH));
       if constexpr (Geo::QV) {
         const uint2 v = quad(tb.v_cent, tb.v_lam, p);
 #pragma unroll
@@ -760,8 +776,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
         const int w = mb / (2 * BPW), r = mb % (2 * BPW), by = r % BPW;
         const uint32_t* s0 = r < BPW ? y0 : z0;
         const uint32_t* s1 = r < BPW ? y1 : z1;
-        const uint2 q0 = lds_table64<kDynSmemBase + Geo::offLV>(bits_at(s0[w], 8 * by, 8, Geo::VSH) | v_lane);
-        const uint2 q1 = lds_table64<kDynSmemBase + Geo::offLV>(bits_at(s1[w], 8 * by, 8, Geo::VSH) | v_lane);
+        const uint2 q0 = lds_table64<kDynSmemBase + Geo::offLV>(quad_index<Geo::IQ, Geo::VSH>(s0[w], by, v_lane));
+        const uint2 q1 = lds_table64<kDynSmemBase + Geo::offLV>(quad_index<Geo::IQ, Geo::VSH>(s1[w], by, v_lane));
         a0 = q0.x;
         a1 = q0.y;
         a2 = q1.x;
@@ -846,8 +862,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
           const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
           uint32_t a0, a1, a2, a3;
           if constexpr (Geo::QK) {  // the byte of channels c0 .. c0+3: one quad per token
-            const uint2 p = lds_table64<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 8, Geo::KSH) | k_lane);
-            const uint2 q = lds_table64<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 8, Geo::KSH) | k_lane);
+            const uint2 p = lds_table64<kDynSmemBase + Geo::offLK>(quad_index<Geo::IQ, Geo::KSH>(kw0[o1 >> 5], (o1 & 31) >> 3, k_lane));
+            const uint2 q = lds_table64<kDynSmemBase + Geo::offLK>(quad_index<Geo::IQ, Geo::KSH>(kw1[o1 >> 5], (o1 & 31) >> 3, k_lane));
             a0 = p.x;
             a1 = q.x;
             a2 = p.y;
