@@ -57,11 +57,11 @@ DECODE_SOURCES = ("tq_internal.cuh", "tq_decode_impl.cuh", "tq_decode.cu", "tq_d
                   "tq_decode_d256.cu", "tq_decode_affine_d64.cu", "tq_decode_affine_d128.cu",
                   "tq_decode_affine_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31446528, "beac15425fddc3fa"),
-    "qjl": (566852096, "beac15425fddc3fa"),
-    "long": (353267200, "beac15425fddc3fa"),
-    "serving": (1102322176, "beac15425fddc3fa"),
-    "affine": (38483456, "beac15425fddc3fa"),
+    "gqa": (31446272, "5604bea35f3a2866"),
+    "qjl": (566628864, "5604bea35f3a2866"),
+    "long": (353745152, "5604bea35f3a2866"),
+    "serving": (1101889536, "5604bea35f3a2866"),
+    "affine": (38483456, "5604bea35f3a2866"),
 }
 
 
@@ -94,10 +94,10 @@ def decode_traffic(workload: str):
 # of active cycles, warp instructions per (token, KV head), warps active %.
 # Keyed, like the traffic, to the digest of the decode sources it describes.
 DECODE_PROFILE: dict[str, tuple[dict, str]] = {
-    "gqa": ({"issue_active_pct": 42.3, "warp_inst_per_token_head": 34.19, "warps_active_pct": 17.5}, "beac15425fddc3fa"),
-    "long": ({"issue_active_pct": 49.3, "warp_inst_per_token_head": 45.72, "warps_active_pct": 12.1}, "beac15425fddc3fa"),
-    "qjl": ({"issue_active_pct": 59.4, "warp_inst_per_token_head": 34.33, "warps_active_pct": 17.2}, "beac15425fddc3fa"),
-    "serving": ({"issue_active_pct": 63.4, "warp_inst_per_token_head": 25.23, "warps_active_pct": 17.1}, "beac15425fddc3fa"),
+    "gqa": ({"issue_active_pct": 41.2, "warp_inst_per_token_head": 33.26, "warps_active_pct": 17.9}, "5604bea35f3a2866"),
+    "long": ({"issue_active_pct": 47.8, "warp_inst_per_token_head": 41.70, "warps_active_pct": 12.2}, "5604bea35f3a2866"),
+    "qjl": ({"issue_active_pct": 58.5, "warp_inst_per_token_head": 33.08, "warps_active_pct": 17.8}, "5604bea35f3a2866"),
+    "serving": ({"issue_active_pct": 61.7, "warp_inst_per_token_head": 23.90, "warps_active_pct": 17.5}, "5604bea35f3a2866"),
 }
 
 

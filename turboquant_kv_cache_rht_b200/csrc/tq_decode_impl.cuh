@@ -227,8 +227,13 @@ struct DecodeGeom {
   static constexpr int kRowB = KB * D / 8;    // bytes of one packed row in global memory
   static constexpr int vRowB = VB * D / 8;
   static constexpr int sRowB = D / 8;
+  // 3-bit keys and 4-bit values at head_dim 128: the PV layout below
+  static constexpr bool PV = D == 128 && KB == 3 && VB == 4 && !AFF;
   static constexpr int KS = k_stride_words(D, KB);
-  static constexpr int VS = v_stride_words(D, VB);
+  // PV with the QJL sketch: value rows unpadded and swizzled (v_row_off);
+  // measured faster than padded rows there, and slower without the sketch
+  static constexpr bool VSW = PV && QJL;
+  static constexpr int VS = VSW ? VB * D / 32 : v_stride_words(D, VB);
   static constexpr int SS = D / 32;
   static constexpr int QB = KB * D / 4;       // key bits per thread quarter (a slice of the row)
   static constexpr int KW = (QB + 31) / 32;   // words of the slice, aligned to bit 0
@@ -249,7 +254,8 @@ struct DecodeGeom {
   static constexpr int EKL = QK ? 3 : 2;               // log2 bytes of a key entry
   static constexpr int EVL = QV ? 3 : 2;               // log2 bytes of a value entry
   // Each table is replicated so that lanes with different (lane mod copies)
-  // never meet in a bank; entry e of copy c sits at byte (e * copies + c) * 4.
+  // never meet in a bank; copy c of entry e sits at byte (e << shift) + c *
+  // (entry bytes), with the entry shift KSH / VSH below.
   // 32 copies (a lane's own) keep every lookup free of bank conflicts; the
   // 4-bit tables of head_dim 256 keep 16 to leave room for the stages
   // (64-bit lookups are served per half-warp, so 16 copies already keep the
@@ -260,8 +266,17 @@ struct DecodeGeom {
   // entry e at byte 256 e and value entry e at 256 e + 128: an index is then
   // the code byte above the lane's copy offset, which one byte permute forms.
   static constexpr bool IQ = QK && QV;
-  static constexpr int KSH = IQ ? 8 : EKL + RKL;  // byte shift of a key entry index
-  static constexpr int VSH = IQ ? 8 : EVL + RVL;  // byte shift of a value entry index
+  // The 3-bit key / 4-bit value shape at head_dim 128 (PV) does the same for
+  // its value pair table (entries 256 bytes apart, 32 copies in the first 128
+  // bytes of each).  The other 128 bytes of every entry form a logical space:
+  // logical offset x sits at byte 128 + x + (x & ~127).  It holds the key pair
+  // table (64 entries of 128 bytes, so key entry e sits at 256 e + 128) and,
+  // after it, the stages' key and value rows and the epilogue's merge buffer.
+  // The map moves every 128-byte block by a multiple of 128 bytes, so an
+  // access keeps the bank it has in a plain layout, and an aligned access of
+  // at most 16 bytes never straddles two blocks.
+  static constexpr int KSH = (IQ || PV) ? 8 : EKL + RKL;  // byte shift of a key entry index
+  static constexpr int VSH = (IQ || PV) ? 8 : EVL + RVL;  // byte shift of a value entry index
   // value quads: y / z bytes per interleaved word (a byte holds two channels)
   static constexpr int BPW = D / 32 < 4 ? D / 32 : 4;
   // affine codec: NG groups of 64 channels, one (scale, bias) word per group
@@ -271,23 +286,47 @@ struct DecodeGeom {
   static constexpr int QBA = 16 * KB;          // key bits per thread quarter and group
   static constexpr int KWA = (QBA + 31) / 32;
   static constexpr int KNWA = (QBA % 32 == 0) ? QBA / 32 : (QBA + 16 + 31) / 32;
-  // one pipeline stage (bytes)
+  // one pipeline stage (bytes): the key and value rows (offsets in the
+  // logical space when PV), then the sign rows and the norms
   static constexpr int offK = 0;
   static constexpr int offV = offK + kDecTile * KS * 4;
-  static constexpr int offS = offV + kDecTile * VS * 4 + 16;
+  static constexpr int kvBytes = offV + kDecTile * VS * 4 + (PV ? 0 : 16);
+  static constexpr int offS = PV ? 0 : kvBytes;
   static constexpr int offKN = offS + (QJL ? kDecTile * SS * 4 : 0);
   static constexpr int offVN = offKN + kDecTile * MB;
   static constexpr int offRN = offVN + kDecTile * MB;
   static constexpr int stage = offRN + (QJL ? kDecTile * 2 : 0);
   static constexpr int stageA = (stage + 127) / 128 * 128;
-  // epilogue merge buffer, reusing the stage area: per warp m[G], l[G], O[G][D]
+  // epilogue merge buffer, reusing the key / value rows of the stages: per
+  // warp m[G], l[G], O[G][D]
   static constexpr int mergeBytes = kDecWarps * G * (D + 2) * 4;
-  static constexpr int stagesBytes =
-      (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
-  // after the stage area
-  static constexpr int offLK = stagesBytes;
-  static constexpr int offLV = IQ ? offLK + 128 : offLK + (LK << KSH);
-  static constexpr int offQ = IQ ? offLK + (LK << 8) : offLV + (LV << VSH);  // float [G][D] rotated query
+  static constexpr int stagesBytes = PV ? kDecStages * stageA
+      : (kDecStages * stageA > mergeBytes ? kDecStages * stageA : (mergeBytes + 127) / 128 * 128);
+  // PV: the tables fill [0, 64 KB); the rows of stage s start at logical
+  // 8192 (s + 1), right after the key table, and the other stage parts after
+  // the table region.  Otherwise the stages come first, then the tables.
+  static constexpr int kvBase = PV ? 128 + 2 * 8192 : 0;             // byte of stage 0's rows
+  static constexpr int kvStride = PV ? 2 * kvBytes : stageA;        // bytes from one stage's rows to the next
+  static constexpr int pBase = PV ? 65536 : 0;                      // byte of stage 0's other parts
+  static constexpr int offLK = PV ? 128 : stagesBytes;
+  static constexpr int offLV = PV ? 0 : IQ ? offLK + 128 : offLK + (LK << KSH);
+  static constexpr int offQ = PV ? pBase + stagesBytes                  // float [G][D] rotated query
+                           : IQ ? offLK + (LK << 8) : offLV + (LV << VSH);
+  // byte of logical offset x (relative to kvBase), and the shift of an
+  // offset by a multiple of 128 bytes
+  __host__ __device__ static constexpr int kvmap(int x) { return PV ? x + (x & ~127) : x; }
+  __host__ __device__ static constexpr int kvshift(int b) { return PV ? 2 * b : b; }
+  // Logical offset of byte 4 w of staged value row r.  Swizzled rows (VSW,
+  // 64 bytes): rows r and r ^ 2 share a 128-byte block (halves (r >> 1) & 1)
+  // and the 16 words of rows with (r >> 2) & 1 set are rotated by 8, so that
+  // rows 2q + c (q = 0..3) of any group of 8 occupy the four (half, rotation)
+  // pairs: a 64-bit read of words 2g, 2g + 1 by lanes (g, q) is free of bank
+  // conflicts.  Otherwise rows are VS words apart.
+  __host__ __device__ static constexpr int v_row_off(int r, int w) {
+    return VSW ? offV + (((r >> 3) << 2) | (((r >> 2) & 1) << 1) | (r & 1)) * 128 + ((r >> 1) & 1) * 64 +
+                     ((w + 8 * ((r >> 2) & 1)) & 15) * 4
+               : offV + r * VS * 4 + w * 4;
+  }
   static constexpr int offQ2 = offQ + G * D * 4;               // float [G][D] QJL query
   static constexpr int offUs = offQ2 + (QJL ? G * D * 4 : 0);  // float [G][NG] group sums (affine)
   static constexpr int offRed = offUs + (AFF ? (G * NG * 4 + 15) / 16 * 16 : 0);  // float scratch
@@ -301,6 +340,11 @@ struct DecodeGeom {
   static constexpr int total = offSched + schedBytes;
   static_assert((KS * 4) % CBK == 0 && (VS * 4) % CBV == 0, "rows aligned to the copy chunk");
   static_assert(VCW <= 4 && VNW <= 4, "value chunk too wide");
+  static_assert(!PV || (kvBytes % 128 == 0 && offV % 128 == 0 && VS == (VSW ? 16 : 20) && LK == 64 && LV == 256 &&
+                        RVL == 5 && VCH == 64 && QB == 96 && KW == 3 && kDecTile % 8 == 0 &&
+                        8192 + kDecStages * kvBytes <= 32768 && mergeBytes <= kDecStages * kvBytes &&
+                        (16 * KS * 4) % 128 == 0 && (8 * KS * 4) % 128 == 0),
+                "PV layout");
 };
 
 // Loads the value chunk of thread group g (bits [g*VCH, (g+1)*VCH)) of one
@@ -378,8 +422,13 @@ __device__ __forceinline__ void value_pairs(const uint32_t (&y)[VCW], const uint
                                             uint32_t lane_off, uint32_t& even, uint32_t& odd) {
   if constexpr (VB == 4) {
     const int w = mb >> 2, k = mb & 3;
-    even = bits_at(y[w], 8 * k, 8, VSH) | lane_off;
-    odd = bits_at(z[w], 8 * k, 8, VSH) | lane_off;
+    if constexpr (VSH == 8) {  // the byte above the lane's copy offset
+      even = __byte_perm(y[w], lane_off, 0x5504u | ((uint32_t)k << 4));
+      odd = __byte_perm(z[w], lane_off, 0x5504u | ((uint32_t)k << 4));
+    } else {
+      even = bits_at(y[w], 8 * k, 8, VSH) | lane_off;
+      odd = bits_at(z[w], 8 * k, 8, VSH) | lane_off;
+    }
   } else if constexpr (VB == 2) {
     const int w = mb >> 3, k = mb & 7;
     even = bits_at(y[w], 4 * k, 4, VSH) | lane_off;
@@ -545,14 +594,14 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   for (int i = 0; i < NK; ++i) {
     const int c = tid + kDecThreads * i, r = c / CK, col = c - r * CK;
     k_row[i] = c < kDecTile * CK ? r : kDecTile;
-    k_dst[i] = Geo::offK + r * Geo::KS * 4 + col * Geo::CBK;
+    k_dst[i] = Geo::kvmap(Geo::offK + r * Geo::KS * 4 + col * Geo::CBK);
     k_src[i] = r * Geo::kRowB + col * Geo::CBK;
   }
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = tid + kDecThreads * i, r = c / CV, col = c - r * CV;
     v_row[i] = c < kDecTile * CV ? r : kDecTile;
-    v_dst[i] = Geo::offV + r * Geo::VS * 4 + col * Geo::CBV;
+    v_dst[i] = Geo::kvmap(Geo::v_row_off(r, col * Geo::CBV / 4));
     v_src[i] = r * Geo::vRowB + col * Geo::CBV;
   }
 #pragma unroll
@@ -562,17 +611,18 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     s_dst[i] = Geo::offS + c * 16;
   }
   auto issue_tile = [&](int stage, int start) {
-    uint8_t* st = smem + stage * Geo::stageA;
+    uint8_t* skv = smem + Geo::kvBase + stage * Geo::kvStride;  // key and value rows
+    uint8_t* st = smem + Geo::pBase + stage * Geo::stageA;       // sign rows and norms
     const int n_valid = min(kDecTile, t_end - start);
     const int rows = (n_valid + 15) & ~15;  // within capacity (a multiple of 16)
     const uint8_t* kb = cv.k_codes + (row_slot + start) * Geo::kRowB;
     const uint8_t* vb = cv.v_codes + (row_slot + start) * Geo::vRowB;
 #pragma unroll
     for (int i = 0; i < NK; ++i)
-      if (k_row[i] < rows) cp_async_chunk<Geo::CBK>(st + k_dst[i], kb + k_src[i]);
+      if (k_row[i] < rows) cp_async_chunk<Geo::CBK>(skv + k_dst[i], kb + k_src[i]);
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-      if (v_row[i] < rows) cp_async_chunk<Geo::CBV>(st + v_dst[i], vb + v_src[i]);
+      if (v_row[i] < rows) cp_async_chunk<Geo::CBV>(skv + v_dst[i], vb + v_src[i]);
     if constexpr (QJL) {
       const uint8_t* sb = cv.k_signs + (row_slot + start) * Geo::sRowB;
 #pragma unroll
@@ -808,7 +858,9 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     if (it + 2 < n_tiles) issue_tile((it + 2) % kDecStages, t_begin + (it + 2) * kDecTile);
     cp_async_commit();
 
-    const uint8_t* st = smem + (it % kDecStages) * Geo::stageA;
+    const int sidx = it % kDecStages;
+    const uint8_t* skv = smem + Geo::kvBase + sidx * Geo::kvStride;  // key and value rows
+    const uint8_t* st = smem + Geo::pBase + sidx * Geo::stageA;       // sign rows and norms
     const int n_valid = min(16, t_end - (t_begin + it * kDecTile + 16 * warp));
     if (n_valid <= 0) continue;
     const int r0 = 16 * warp;  // the warp's slab: rows r0 .. r0+15 of the stage
@@ -818,11 +870,40 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     // latency overlaps the score work
     uint32_t va[Geo::VCW], vb2[Geo::VCW], vc[Geo::VCW], vd[Geo::VCW];
     {
-      const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Geo::offV) + (r0 + 2 * qd) * Geo::VS;
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow, g, va);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + Geo::VS, g, vb2);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
-      load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
+      if constexpr (Geo::PV) {
+        // words 2g, 2g + 1 of rows 2q, 2q + 1, 2q + 8, 2q + 9 of the slab, as
+        // mapped 8-byte pieces (an aligned piece never straddles two blocks)
+        uint2 x0, x1, x2, x3;
+        if constexpr (Geo::VSW) {  // the rows sit 128, 512, 640 logical bytes after the first
+          const uint8_t* v0 = skv + Geo::kvshift(Geo::v_row_off(r0, 0) - Geo::offV) +
+                              Geo::kvmap(Geo::v_row_off(2 * qd, 2 * g));
+          static_assert(!Geo::VSW || (Geo::v_row_off(1, 0) - Geo::v_row_off(0, 0) == 128 &&
+                                      Geo::v_row_off(8, 0) - Geo::v_row_off(0, 0) == 512), "value row blocks");
+          x0 = *reinterpret_cast<const uint2*>(v0);
+          x1 = *reinterpret_cast<const uint2*>(v0 + Geo::kvshift(128));
+          x2 = *reinterpret_cast<const uint2*>(v0 + Geo::kvshift(512));
+          x3 = *reinterpret_cast<const uint2*>(v0 + Geo::kvshift(640));
+        } else {  // padded rows: rows 2q and 2q + 1 mapped separately, + 8 rows = whole blocks
+          const uint8_t* v0 = skv + Geo::kvshift(r0 * Geo::VS * 4);
+          const int o0 = Geo::kvmap(Geo::v_row_off(2 * qd, 2 * g));
+          const int o1 = Geo::kvmap(Geo::v_row_off(2 * qd + 1, 2 * g));
+          constexpr int R8 = Geo::kvshift(8 * Geo::VS * 4);
+          x0 = *reinterpret_cast<const uint2*>(v0 + o0);
+          x1 = *reinterpret_cast<const uint2*>(v0 + o1);
+          x2 = *reinterpret_cast<const uint2*>(v0 + o0 + R8);
+          x3 = *reinterpret_cast<const uint2*>(v0 + o1 + R8);
+        }
+        va[0] = x0.x; va[1] = x0.y;
+        vb2[0] = x1.x; vb2[1] = x1.y;
+        vc[0] = x2.x; vc[1] = x2.y;
+        vd[0] = x3.x; vd[1] = x3.y;
+      } else {
+        const uint32_t* vrow = reinterpret_cast<const uint32_t*>(skv + Geo::offV) + (r0 + 2 * qd) * Geo::VS;
+        load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow, g, va);
+        load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + Geo::VS, g, vb2);
+        load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 8 * Geo::VS, g, vc);
+        load_value_chunk<Geo::VCH, Geo::VCW, Geo::VNW>(vrow + 9 * Geo::VS, g, vd);
+      }
     }
     uint32_t vsab = 0u, vbab = 0u, vscd = 0u, vbcd = 0u;
     if constexpr (AFF) {
@@ -854,9 +935,22 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
           for (int e = 0; e < 4; ++e) sacc[par][j][e] = 0.f;
       {
         uint32_t kw0[Geo::KW], kw1[Geo::KW];
-        const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
-        load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);  // bits of quarter qd, tokens g
-        load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);  // and g + 8
+        if constexpr (Geo::PV) {
+          // words 3 qd .. 3 qd + 2 of rows g and g + 8, each mapped (a row may
+          // straddle two 128-byte blocks)
+          const uint8_t* k0 = skv + Geo::kvshift(r0 * Geo::KS * 4);
+          constexpr int R8 = Geo::kvshift(8 * Geo::KS * 4);
+#pragma unroll
+          for (int i = 0; i < Geo::KW; ++i) {
+            const int o = Geo::kvmap(Geo::offK + g * Geo::KS * 4 + (Geo::KW * qd + i) * 4);
+            kw0[i] = *reinterpret_cast<const uint32_t*>(k0 + o);
+            kw1[i] = *reinterpret_cast<const uint32_t*>(k0 + o + R8);
+          }
+        } else {
+          const uint32_t* k0 = reinterpret_cast<const uint32_t*>(skv + Geo::offK) + (r0 + g) * Geo::KS;
+          load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);  // bits of quarter qd, tokens g
+          load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);  // and g + 8
+        }
 #pragma unroll
         for (int kb = 0; kb < Geo::KBLK; ++kb) {
           const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;  // code pairs (c0,c0+1) and (c0+2,c0+3)
@@ -898,7 +992,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
           for (int e = 0; e < 4; ++e) sacc[gg][j][e] = 0.f;
       uint32_t kw0[Geo::NG][Geo::KWA], kw1[Geo::NG][Geo::KWA];
-      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st + Geo::offK) + (r0 + g) * Geo::KS;
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(skv + Geo::offK) + (r0 + g) * Geo::KS;
 #pragma unroll
       for (int gg = 0; gg < Geo::NG; ++gg) {
         load_value_chunk<Geo::QBA, Geo::KWA, Geo::KNWA>(k0 + gg * 2 * KB, qd, kw0[gg]);
@@ -1083,22 +1177,23 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     l_part[j] = l;
   }
   __syncthreads();  // every warp is done with the stages (no copies are in flight)
-  float* mw = reinterpret_cast<float*>(smem);  // [warp][G]
-  float* lw = mw + kDecWarps * G;              // [warp][G]
-  float* ow = lw + kDecWarps * G;              // [warp][G][D]
+  // merge buffer over the stages' key / value rows: m[warp][G], l[warp][G],
+  // O[warp][G][D] (floats; float i at logical byte 4 i)
+  auto mrg = [&](int i) -> float& { return *reinterpret_cast<float*>(smem + Geo::kvBase + Geo::kvmap(4 * i)); };
+  constexpr int LW = kDecWarps * G, OW = 2 * kDecWarps * G;
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     const int head = 4 * j + qd;
     if (head < G) {
       if (g == 0) {
-        mw[warp * G + head] = m_run[j];
-        lw[warp * G + head] = l_part[j];
+        mrg(warp * G + head) = m_run[j];
+        mrg(LW + warp * G + head) = l_part[j];
       }
-      float* o = ow + (warp * G + head) * D + g * (D / 8);
+      const int o = OW + (warp * G + head) * D + g * (D / 8);
 #pragma unroll
       for (int mb = 0; mb < Geo::MBLK; ++mb) {
-        o[value_channel<Geo::QV, Geo::BPW>(mb, 0)] = acc[j][mb][0] + acc[j][mb][1];
-        o[value_channel<Geo::QV, Geo::BPW>(mb, 1)] = acc[j][mb][2] + acc[j][mb][3];
+        mrg(o + value_channel<Geo::QV, Geo::BPW>(mb, 0)) = acc[j][mb][0] + acc[j][mb][1];
+        mrg(o + value_channel<Geo::QV, Geo::BPW>(mb, 1)) = acc[j][mb][2] + acc[j][mb][3];
       }
     }
   }
@@ -1107,10 +1202,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
   float* wt = reinterpret_cast<float*>(smem + Geo::offRed);   // [warp][G] merge weights
   if (tid < kDecWarps * G) {
     const int w = tid / G, h = tid % G;
-    float M = mw[h];
+    float M = mrg(h);
 #pragma unroll
-    for (int v = 1; v < kDecWarps; ++v) M = fmaxf(M, mw[v * G + h]);
-    const float m = mw[w * G + h];
+    for (int v = 1; v < kDecWarps; ++v) M = fmaxf(M, mrg(v * G + h));
+    const float m = mrg(w * G + h);
     wt[tid] = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
     if (w == 0) red[kDecWarps * G + h] = M;
   }
@@ -1122,13 +1217,13 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
     const int h = i / D, ch = i % D;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) v = fmaf(ow[(w * G + h) * D + ch], wt[w * G + h], v);
+    for (int w = 0; w < kDecWarps; ++w) v = fmaf(mrg(OW + (w * G + h) * D + ch), wt[w * G + h], v);
     dst_o[i] = v;
   }
   if (tid < G) {
     float l = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) l = fmaf(lw[w * G + tid], wt[w * G + tid], l);
+    for (int w = 0; w < kDecWarps; ++w) l = fmaf(mrg(LW + w * G + tid), wt[w * G + tid], l);
     dst_ml[2 * tid] = red[kDecWarps * G + tid];
     dst_ml[2 * tid + 1] = l;
   }
