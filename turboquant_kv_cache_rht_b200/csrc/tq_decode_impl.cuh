@@ -262,10 +262,11 @@ struct DecodeGeom {
   // quad tables free of conflicts)
   static constexpr int RKL = QK ? 4 : (KB <= 3 || D <= 128) ? 5 : 4;  // log2 key copies
   static constexpr int RVL = QV ? 4 : (VB <= 3 || D <= 128) ? 5 : 4;  // log2 value copies
-  // When both tables are quads their 128-byte entries are interleaved, key
-  // entry e at byte 256 e and value entry e at 256 e + 128: an index is then
-  // the code byte above the lane's copy offset, which one byte permute forms.
-  static constexpr bool IQ = QK && QV;
+  // When both tables are quads, or both are 4-bit pair tables of 32 copies,
+  // their 128-byte entries are interleaved, key entry e at byte 256 e and
+  // value entry e at 256 e + 128: an index is then the code byte above the
+  // lane's copy offset, which one byte permute forms.
+  static constexpr bool IQ = (QK && QV) || (KB == 4 && VB == 4 && RKL == 5 && RVL == 5);
   // The 3-bit key / 4-bit value shape at head_dim 128 (PV) does the same for
   // its value pair table (entries 256 bytes apart, 32 copies in the first 128
   // bytes of each).  The other 128 bytes of every entry form a logical space:
@@ -371,9 +372,10 @@ __device__ __forceinline__ uint32_t bits_at(uint32_t x, int pos, int width, int 
   return pos >= scale ? (x >> (pos - scale)) & mask : (x << (scale - pos)) & mask;
 }
 
-// Index of the quad-table entry of byte `by` of x for a lane whose copy offset
-// is lane_off (< 256): with the interleaved layout (entry shift 8) the byte
-// permute places the code byte above the offset in one instruction.
+// Index of the table entry named by byte `by` of x (a quad, or a pair of 4-bit
+// codes) for a lane whose copy offset is lane_off (< 256): with an entry shift
+// of 8 the byte permute places the code byte above the offset in one
+// instruction.
 template <bool IQ, int SH>
 __device__ __forceinline__ uint32_t quad_index(uint32_t x, int by, uint32_t lane_off) {
   if constexpr (IQ) {
@@ -486,12 +488,15 @@ __device__ __forceinline__ long long block_exclusive_scan(long long x, long long
 // CTAs per SM the register budget is sized for: d <= 128 fits three CTAs
 // (168 registers: measured faster than four CTAs at 128, where the kernel
 // spends instructions on register moves), two when the shape carries two
-// column tiles and the QJL sketch; d = 256 fits two.
-template <int D, int G, bool QJL>
-constexpr int decode_min_ctas() { return D <= 128 ? ((G > 4 && QJL) ? 2 : 3) : 2; }
+// column tiles and the QJL sketch, or when its shared memory (B200: 228 KB per
+// SM, 1 KB reserved per CTA) holds only two; d = 256 fits two.
+template <int D, int G, int KB, int VB, bool QJL, bool AFF>
+constexpr int decode_min_ctas() {
+  return D <= 128 && !(G > 4 && QJL) && 3 * (DecodeGeom<D, G, KB, VB, QJL, AFF>::total + 1024) <= 228 * 1024 ? 3 : 2;
+}
 
 template <int D, int G, int KB, int VB, bool QJL, bool AFF>
-__global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
+__global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, KB, VB, QJL, AFF>())
     decode_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                   const void* __restrict__ q, int q_dtype, int q_heads, float scale_log2,
                   int max_ctx, int nslots, float* __restrict__ ws) {
@@ -963,10 +968,17 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
             a2 = p.y;
             a3 = q.y;
           } else {
-            a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
-            a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
-            a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
-            a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+            if constexpr (Geo::IQ) {  // 4-bit pairs: whole bytes
+              a0 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw0[o1 >> 5], (o1 & 31) >> 3, k_lane));
+              a1 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw1[o1 >> 5], (o1 & 31) >> 3, k_lane));
+              a2 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw0[o2 >> 5], (o2 & 31) >> 3, k_lane));
+              a3 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw1[o2 >> 5], (o2 & 31) >> 3, k_lane));
+            } else {
+              a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+              a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane);
+              a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+              a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane);
+            }
           }
 #pragma unroll
           for (int j = 0; j < NT; ++j) mma16816(sacc[kb & 1][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
@@ -1001,10 +1013,18 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, QJL>())
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int gg = kb >> 2, o1 = KB * 4 * (kb & 3), o2 = o1 + 2 * KB;
-        const uint32_t a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
-        const uint32_t a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
-        const uint32_t a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
-        const uint32_t a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
+        uint32_t a0, a1, a2, a3;
+        if constexpr (Geo::IQ) {  // 4-bit pairs: whole bytes
+          a0 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw0[gg][o1 >> 5], (o1 & 31) >> 3, k_lane));
+          a1 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw1[gg][o1 >> 5], (o1 & 31) >> 3, k_lane));
+          a2 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw0[gg][o2 >> 5], (o2 & 31) >> 3, k_lane));
+          a3 = lds_table<kDynSmemBase + Geo::offLK>(quad_index<true, 8>(kw1[gg][o2 >> 5], (o2 & 31) >> 3, k_lane));
+        } else {
+          a0 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
+          a1 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o1, 2 * KB, Geo::KSH) | k_lane);
+          a2 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw0[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
+          a3 = lds_table<kDynSmemBase + Geo::offLK>(field_scaled(kw1[gg], Geo::KWA, o2, 2 * KB, Geo::KSH) | k_lane);
+        }
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma16816(sacc[gg][j], a0, a1, a2, a3, bk[j][kb][0], bk[j][kb][1]);
       }

@@ -42,13 +42,22 @@ constexpr int kAppendWarps = 8;
 constexpr int kBulkE = 32;
 
 // The codec of one vector at its code width: Lloyd-Max (norm, codes, sketch)
-// or the affine group-64 comparison codec (scale/bias pairs in `norm`).
-template <int D, int E, bool AFF>
+// or the affine group-64 comparison codec (scale/bias pairs in `norm`).  BITS
+// fixes the width at compile time (a grid of one kind: a third less register
+// pressure than the kernel that holds all three widths, so a third more warps
+// per SM); 0 takes it from `bits`.
+template <int D, int E, bool AFF, int BITS = 0>
 __device__ __forceinline__ void encode_vector(int bits, float (&u)[E], const Tables& tb, bool is_v,
                                               int g, int lane, bool valid, uint8_t* codes,
                                               uint16_t* norm, uint8_t* signs, uint16_t* rnorm,
                                               const float* s_kcent) {
-  if constexpr (AFF) {
+  if constexpr (BITS != 0) {
+    if constexpr (AFF)
+      encode_affine_store<D, E, BITS>(u, tb, is_v, g, lane, valid, codes,
+                                      reinterpret_cast<uint32_t*>(norm), signs, rnorm);
+    else
+      encode_store<D, E, BITS>(u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
+  } else if constexpr (AFF) {
     uint32_t* meta = reinterpret_cast<uint32_t*>(norm);
     if (bits == 2)
       encode_affine_store<D, E, 2>(u, tb, is_v, g, lane, valid, codes, meta, signs, rnorm);
@@ -77,7 +86,7 @@ constexpr int kAppendThreads = 32 * kAppendWarps;
 // bulk append runs keys and values as two grids, so that each grid executes
 // one code width and its unrolled code stays in the instruction cache; the
 // second grid publishes).
-template <int D, typename T, int E, bool AFF, bool BULK>
+template <int D, typename T, int E, bool AFF, bool BULK, int BITS = 0>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_append_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                            const T* __restrict__ kin, const T* __restrict__ vin, int n_new,
@@ -124,7 +133,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
-    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
+    encode_vector<D, E, AFF, BITS>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
   }
 
   // The last block of this batch row to finish publishes the new length.  Every
@@ -149,7 +158,7 @@ __global__ void __launch_bounds__(kAppendThreads)
 // smaller one (a [batch][T][heads][d] cache) and with h outermost otherwise,
 // so consecutive lanes read consecutive memory.  Without `lengths` every row
 // holds max_len vectors and no length or flag is written.
-template <int D, typename T, int E, bool AFF>
+template <int D, typename T, int E, bool AFF, int BITS = 0>
 __global__ void __launch_bounds__(kAppendThreads)
     quantize_convert_kernel(const __grid_constant__ Tables tb, const __grid_constant__ CacheView cv,
                             const T* __restrict__ kin, const T* __restrict__ vin, long stride_b,
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     uint16_t* norm = (is_v ? cv.v_norm : cv.k_norm) + slot * NH;
     uint8_t* signs = (!is_v && tb.qjl) ? cv.k_signs + slot * (long)(D / 8) : nullptr;
     uint16_t* rnorm = (!is_v && tb.qjl) ? cv.k_rnorm + slot : nullptr;
-    encode_vector<D, E, AFF>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
+    encode_vector<D, E, AFF, BITS>(bits, u, tb, is_v, g, lane, valid, codes, norm, signs, rnorm, s_kcent);
   }
   pdl_trigger();
 }
@@ -235,9 +244,15 @@ cudaError_t launch_layout(const Tables& tb, const CacheView& cv, const void* k, 
     return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 1);
   } else {
     cfg.gridDim = dim3((unsigned)blocks_per_kind, (unsigned)cv.batch);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 0);
+    auto of_width = [](int bits) {  // the kernel of one code width
+      return bits == 2 ? quantize_append_kernel<D, T, E, AFF, BULK, 2>
+           : bits == 3 ? quantize_append_kernel<D, T, E, AFF, BULK, 3>
+                       : quantize_append_kernel<D, T, E, AFF, BULK, 4>;
+    };
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, of_width(tb.k_bits), tb, cv, kp, vp, n_new, (int)blocks_per_kind, 0, 0);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, n_new, (int)blocks_per_kind, 1, 1);
+    return cudaLaunchKernelEx(&cfg, of_width(tb.v_bits), tb, cv, kp, vp, n_new, (int)blocks_per_kind, 1, 1);
   }
 }
 
@@ -278,10 +293,19 @@ cudaError_t launch_convert_layout(const Tables& tb, const CacheView& cv, const v
   // as for the append)
   const bool split = !small && kinds == 2;
   cfg.gridDim = dim3((unsigned)((split ? 1 : kinds) * blocks_per_kind), (unsigned)cv.batch);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
+  if (!split) {
+    return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
+                              (int)blocks_per_kind, heads_inner, 0);
+  }
+  auto of_width = [](int bits) {  // the kernel of one code width
+    return bits == 2 ? quantize_convert_kernel<D, T, E, AFF, 2>
+         : bits == 3 ? quantize_convert_kernel<D, T, E, AFF, 3>
+                     : quantize_convert_kernel<D, T, E, AFF, 4>;
+  };
+  cudaError_t e = cudaLaunchKernelEx(&cfg, of_width(tb.k_bits), tb, cv, kp, vp, sb, sh, st, lengths, max_len,
                                      (int)blocks_per_kind, heads_inner, 0);
-  if (e != cudaSuccess || !split) return e;
-  return cudaLaunchKernelEx(&cfg, kern, tb, cv, kp, vp, sb, sh, st, lengths, max_len,
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, of_width(tb.v_bits), tb, cv, kp, vp, sb, sh, st, lengths, max_len,
                             (int)blocks_per_kind, heads_inner, 1);
 }
 
