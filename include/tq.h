@@ -205,10 +205,14 @@ tq_status tq_quantize_cache(const tq_codebook* cb, const tq_cache* cache, const 
                             const void* v, tq_dtype dtype, int64_t stride_b, int64_t stride_h,
                             int64_t stride_t, const int32_t* lengths, int max_len, void* stream);
 
-/* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes):
- * (min(592, U * ceil(max_ctx / 64)) + U - 1) * (q_heads / kv_heads) *
- * (head_dim + 2) * 4, U = batch * kv_heads -- one partial result per (CTA,
- * unit) the decode's work partition can produce. */
+/* Workspace bytes tq_decode_attention needs for these sizes (0 on bad sizes).
+ * Size workspaces by calling this function: the figure follows the decode
+ * kernel's grid and may change with the library version.  For information,
+ * this version returns (min(592, U * ceil(max_ctx / 64)) + U - 1) *
+ * (q_heads / kv_heads) * (head_dim + 2) * 4 with U = batch * kv_heads: one
+ * partial result per (CTA, unit) the work partition can produce, for grids of
+ * at most 592 CTAs (4 per SM on 148 SMs).  It depends on the sizes alone, so
+ * one workspace serves every call (and every captured graph) of those sizes. */
 size_t tq_decode_workspace_bytes(const tq_codebook* cb, int batch, int q_heads, int kv_heads,
                                  int max_ctx);
 
