@@ -256,11 +256,10 @@ tq_status tq_decode_attention(const tq_codebook* cb, const tq_cache* cache, cons
  *     library routine is called.
  *   - A decode whose scratch (tq_decode_workspace_bytes for the same sizes)
  *     exceeds 8 MiB is rejected with TQ_ERR_CAPACITY and enqueues nothing.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.  The cached address belongs to the device's primary
- *     context: after a reset of that context (cudaDeviceReset) the library
- *     must be unloaded and loaded again before this entry point is called.
+ *   - Every call looks up the array's address in the current context (no
+ *     allocation), so a reset of the context (cudaDeviceReset) needs nothing
+ *     special; the first call on a device loads the array's module, so make
+ *     it before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Nothing in it needs to start at zero (every partial is written before
  *     it is read), but calls that overlap on the GPU (different streams, or

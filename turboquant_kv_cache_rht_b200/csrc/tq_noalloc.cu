@@ -13,7 +13,6 @@
 #include "tq_internal.cuh"
 
 #include <cstdio>
-#include <mutex>
 
 namespace {
 
@@ -24,33 +23,21 @@ namespace {
 constexpr size_t kScratchBytes = 8u << 20;
 static __device__ __align__(256) float g_decode_scratch[kScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device.  On the host the
-// array's name only stands in for the symbol, so the address is looked up
-// once per device (with that device current) and cached.
+// Device address of g_decode_scratch in the current context.  On the host the
+// array's name only stands in for the symbol, so the address is looked up on
+// every call: the lookup allocates nothing and costs little once the module is
+// loaded, and it stays right after the context is reset (the module, and with
+// it the array, is loaded afresh into the new context).
 tq_status scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess)
-    return (tq_status)tq::record_error(TQ_ERR_CUDA, cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices)
-    return (tq_status)tq::record_error(TQ_ERR_UNSUPPORTED, "device ordinal out of range");
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || !p) {
-      char msg[256];
-      std::snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static decode scratch failed: %s",
-                    cudaGetErrorString(e));
-      return (tq_status)tq::record_error(TQ_ERR_CUDA, msg);
-    }
-    g_scratch_ptr[dev] = p;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || !p) {
+    char msg[256];
+    std::snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static decode scratch failed: %s",
+                  cudaGetErrorString(e));
+    return (tq_status)tq::record_error(TQ_ERR_CUDA, msg);
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return TQ_OK;
 }
 
