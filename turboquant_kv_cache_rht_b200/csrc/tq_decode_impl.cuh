@@ -17,11 +17,16 @@
 //   scores  S[token][col]  = K_hat[token][ch] . Qt[ch][col]
 //   output  O^T[ch][col]  += V_hat^T[ch][token] . P^T[token][col]
 // where a column is (head, part): the query and the probabilities are split
-// into fp16 hi + lo parts, so their products carry about 22 bits.  Key values
-// are split the same way (centroid = hi + lo, both fp16); value centroids are
-// used at fp16 precision.  The packed codes never become a dequantized
-// cache: each thread turns its own code bits into MMA fragment registers
-// through small pair tables (two codes -> two fp16 values) in shared memory.
+// into fp16 hi + lo parts, so their products carry about 22 bits.  Key and
+// value centroids enter as single fp16 values of lambda * c, with a per-table
+// scale lambda in [1, 2) chosen on the host so that these roundings are
+// nearly exact (lambda is divided out in fp32).  The packed codes never
+// become a dequantized cache: each thread turns its own code bits into MMA
+// fragment registers through small tables in shared memory (pairs: two codes
+// -> two fp16 values; quads: a byte of four 2-bit codes -> four), replicated
+// so that a warp's lookups never share a bank.  Where a table index is a
+// whole code byte, the tables' entries are 256 bytes apart and one byte
+// permute forms the index (see DecodeGeom).
 //
 // The MMA reduction order is free, so channels are assigned to fragment
 // slots such that every thread reads one contiguous slice of each packed row:
