@@ -296,8 +296,8 @@ def tq_decode_attention(cb: Codebook, cache: Cache, q: torch.Tensor, out: torch.
     max_ctx = cache.capacity if max_ctx is None else max_ctx
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-    need = tq_decode_workspace_bytes(cb, cache.batch, hq, cache.kv_heads, max_ctx)
-    if workspace is None:
+    if workspace is None:   # (the library checks a caller's workspace size itself)
+        need = tq_decode_workspace_bytes(cb, cache.batch, hq, cache.kv_heads, max_ctx)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     cs = cache.struct()
     _check(lib.tq_decode_attention(cb.handle, C.byref(cs), q.data_ptr(), _dtype_code(q), hq,
