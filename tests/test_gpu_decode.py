@@ -81,14 +81,20 @@ def test_gqa_groups_head_dim_64(G, qjl):
     assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
 
 
+# Every group size on the table layouts of head_dim 128: 3-bit keys / 4-bit
+# values (value table indexed by a byte permute, staged rows in the tables'
+# second halves; padded rows without the sketch, swizzled rows with it), and
+# the interleaved 4-bit pair and 2-bit quad tables.
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-def test_gqa_groups(G):
+@pytest.mark.parametrize("kb,vb,qjl", [(3, 4, True), (3, 4, False), (4, 4, False), (2, 2, True)])
+def test_gqa_groups(G, kb, vb, qjl):
     d, B, Hkv = 128, 1, 2
     lengths = [517]
-    cb, cache, k, v, q = _setup(d, 3, 4, True, B, Hkv, G, lengths, 528, seed=G, corr=True)
+    seed = G + 10 * kb + vb + 100 * qjl
+    cb, cache, k, v, q = _setup(d, kb, vb, qjl, B, Hkv, G, lengths, 528, seed=seed, corr=True)
     out = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=528)
     torch.cuda.synchronize()
-    ref = _oracle(d, 3, 4, True, G, k, v, q, lengths, G)
+    ref = _oracle(d, kb, vb, qjl, seed, k, v, q, lengths, G)
     assert_rows_close(out.cpu().numpy().reshape(-1, d), ref.reshape(-1, d))
 
 
