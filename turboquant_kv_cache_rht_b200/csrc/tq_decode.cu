@@ -33,10 +33,10 @@ constexpr int kMaxParts = 1024;  // partials one unit can have (at most one per 
 static_assert(kMaxTargetCtas <= kMaxParts, "a unit's partials must fit the merge");
 
 // Merges the partial results of one (query head, batch row) and applies the
-// inverse rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / d with
-// w_s = 2^(m_s - max m) ("How to Use TurboQuant ...", "What is TurboQuant?":
-// _rht_inverse; the 1/d collects the rotation's and the dequantization's
-// 1/sqrt(d)).  The affine codec's values are not rotated: o = sum / l.  The
+// inverse rotation: o = D1 H (sum_s w_s o_s) / (sum_s w_s l_s) / (d v_lam)
+// with w_s = 2^(m_s - max m) ("How to Use TurboQuant ...", "What is
+// TurboQuant?": _rht_inverse; the 1/d collects the rotation's and the
+// dequantization's 1/sqrt(d), and v_lam is the value table's scale).  The affine codec's values are not rotated: o = sum / l.  The
 // partials are those of the CTAs whose tile ranges meet the unit's (the
 // partition of DecodePlan, recomputed here from the lengths).
 // Every partial is loaded at once (warp w takes partials w, w+8, ..., lane l

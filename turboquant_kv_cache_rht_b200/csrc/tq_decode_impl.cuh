@@ -518,9 +518,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, KB, VB, QJL
     if (tid == 0) atomicOr(cv.status, (int)kFlagLayout);
     return;
   }
-  // ---- pair tables (two codes -> an fp16 pair) of the keys and of the
-  //      values, each centroid scaled by its table's k_lam / v_lam so that
-  //      its fp16 rounding is nearly exact.  They depend on the kernel
+  // ---- code tables of the keys and of the values (pairs: two codes -> an
+  //      fp16 pair; quads: a byte of four 2-bit codes -> four fp16 values),
+  //      each centroid scaled by its table's k_lam / v_lam so that its fp16
+  //      rounding is nearly exact.  They depend on the kernel
   //      parameters alone, so they are built before the wait, overlapping the
   //      previous kernel in the stream.
   {
