@@ -20,7 +20,12 @@ read by the decode, queries, outputs, appended K/V and their codes) / device
 time, in GB/s, plus ctx-tokens/s, the decode call's roofline against the
 measured HBM copy bandwidth, bulk quantize Mvec/s, an end-to-end figure through
 host buffers, the FP16/BF16 dense decode baselines on the same GPU, and the CPU
-oracle timed on the host as a baseline.
+oracle timed on the host as a baseline.  The default workload is `serving`
+(32 ragged rows of 8k-64k tokens); the line also carries `long_context`: the
+decode calls of the 131k-token `qjl` and 524k-token `long` workloads with their
+own roofline fractions and dense baselines.  `roofline.traffic` (ncu DRAM
+bytes) and `roofline.issue` (issue utilisation) come from committed ncu
+summaries and read null once the decode sources differ from the captured ones.
 
 With several GPUs (torchrun) every rank runs an independent replica of the
 workload ("replicas only": the path has no exchange step); `value` is the sum
