@@ -16,7 +16,8 @@
 // The second takes 128 weight rows and 4 or 8 inputs per CTA; per block it
 // stages the rows' codes, their norms and the block's input fragments with
 // one 3-stage cp.async pipeline, and each warp scores 2 slabs of 16 rows with
-// the decode's pair table and hi/lo split.  When rows x inputs give too few
+// a pair table as the decode's keys use (two codes -> an fp16 pair of
+// lambda-scaled centroids, 32 copies), one MMA per 16 rows and k-block.  When rows x inputs give too few
 // CTAs, the blocks are split across CTAs and the partial sums are merged in a
 // fixed order.
 #include "tq_decode_impl.cuh"
@@ -46,8 +47,8 @@ struct MmGeom {
   static constexpr int KW = (QB + 31) / 32;
   static constexpr int KNW = (QB % 32 == 0) ? QB / 32 : (QB + 16 + 31) / 32;
   static constexpr int LK = 1 << (2 * KB);
-  static constexpr int RKL = KB <= 3 ? 4 : 3;
-  static constexpr int KSH = 3 + RKL;
+  static constexpr int RKL = 5;        // 32 copies: a warp's lookups never share a bank
+  static constexpr int KSH = 2 + RKL;  // 4-byte entries
   static constexpr int FW = frag_words<D, NT>();
   // one stage: codes [kMmRows][KS], norms [kMmRows], fragments [FW], scales [4 NT]
   static constexpr int offN = kMmRows * KS * 4;
@@ -55,7 +56,7 @@ struct MmGeom {
   static constexpr int offS = offF + FW * 4;
   static constexpr int stageA = (offS + 16 * NT + 127) / 128 * 128;
   static constexpr int offLK = kMmStages * stageA;
-  static constexpr int total = offLK + (LK << RKL) * 8;
+  static constexpr int total = offLK + (LK << KSH);
 };
 
 // Input rotation: one warp per (input, block).  frag[(j * groups + cg) * FW ..]
@@ -127,18 +128,16 @@ __global__ void __launch_bounds__(kMmThreads)
   const int row0 = blockIdx.x * kMmRows, cg = blockIdx.y, split = blockIdx.z;
   const int j0 = split * blocks_per_split, j1 = min(nblocks, j0 + blocks_per_split);
 
-  // key pair table (hi pair, lo pair), as in the decode; kernel parameters only
+  // pair table of fp16(k_lam * c) (k_lam divided out with the scales); it
+  // depends on the kernel parameters only, so it is built before the wait
   {
     constexpr int RK = 1 << Geo::RKL;
     for (int p = tid; p < Geo::LK; p += kMmThreads) {
-      const float ca = tb.k_cent[p & ((1 << KB) - 1)], cb = tb.k_cent[p >> KB];
-      const __half ha = __float2half_rn(ca), hb = __float2half_rn(cb);
-      const __half la = __float2half_rn(ca - __half2float(ha));
-      const __half lb = __float2half_rn(cb - __half2float(hb));
-      const uint32_t hi = pack_half2(ha, hb), lo = pack_half2(la, lb);
-      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK) + p * (RK / 2);
+      const uint32_t v = pack_half2(__float2half_rn(tb.k_cent[p & ((1 << KB) - 1)] * tb.k_lam),
+                                    __float2half_rn(tb.k_cent[p >> KB] * tb.k_lam));
+      uint4* dst = reinterpret_cast<uint4*>(smem + Geo::offLK + (p << Geo::KSH));
 #pragma unroll
-      for (int c = 0; c < RK / 2; ++c) dst[c] = make_uint4(hi, lo, hi, lo);
+      for (int c = 0; c < RK / 4; ++c) dst[c] = make_uint4(v, v, v, v);
     }
   }
   pdl_wait();
@@ -171,7 +170,8 @@ __global__ void __launch_bounds__(kMmThreads)
   cp_async_commit();
 
   const uint8_t* lutK = smem + Geo::offLK;
-  const uint32_t k_lane = (uint32_t)(lane & ((1 << Geo::RKL) - 1)) << 3;
+  const uint32_t k_lane = (uint32_t)lane << 2;
+  const float inv_lam = 1.0f / tb.k_lam;
   float y[kMmSlabs][NT][2];  // rows (slab, g) and (slab, g + 8), input cg*CPG + 4 nt + qd
 #pragma unroll
   for (int s = 0; s < kMmSlabs; ++s)
@@ -198,20 +198,22 @@ __global__ void __launch_bounds__(kMmThreads)
           bk[nt][kb][0] = v.x;
           bk[nt][kb][1] = v.y;
         }
-        post[nt] = sc[4 * nt + qd];
+        post[nt] = sc[4 * nt + qd] * inv_lam;
       }
     }
 #pragma unroll
     for (int s = 0; s < kMmSlabs; ++s) {
       const int r0 = 16 * (warp * kMmSlabs + s);
       if (r0 >= valid_rows) break;
-      float sacc[2][NT][4], sacc2[2][NT][4];
+      // MMA rows g and g + 8 are weight rows r0 + g and r0 + g + 8; columns
+      // are (input, part): input qd's fp16 hi and lo parts at 2 qd, 2 qd + 1
+      float sacc[2][NT][4];
 #pragma unroll
       for (int par = 0; par < 2; ++par)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[par][nt][e] = sacc2[par][nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) sacc[par][nt][e] = 0.f;
       uint32_t kw0[Geo::KW], kw1[Geo::KW];
       const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st) + (r0 + g) * Geo::KS;
       load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);
@@ -219,26 +221,21 @@ __global__ void __launch_bounds__(kMmThreads)
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;
-        const uint2 p0 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p1 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p2 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint2 p3 = *reinterpret_cast<const uint2*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma16816(sacc[kb & 1][nt], p0.x, p0.y, p1.x, p1.y, bk[nt][kb][0], bk[nt][kb][1]);
-          mma16816(sacc2[kb & 1][nt], p2.x, p2.y, p3.x, p3.y, bk[nt][kb][0], bk[nt][kb][1]);
-        }
+        for (int nt = 0; nt < NT; ++nt) mma16816(sacc[kb & 1][nt], a0, a1, a2, a3, bk[nt][kb][0], bk[nt][kb][1]);
       }
       const uint16_t* nr = reinterpret_cast<const uint16_t*>(st + Geo::offN) + r0;
       const float n0 = __half2float(__ushort_as_half(nr[g]));
       const float n1 = __half2float(__ushort_as_half(nr[g + 8]));
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        y[s][nt][0] = fmaf(((sacc[0][nt][0] + sacc[1][nt][0]) + (sacc[0][nt][1] + sacc[1][nt][1])) +
-                               ((sacc[0][nt][2] + sacc[1][nt][2]) + (sacc[0][nt][3] + sacc[1][nt][3])),
+        y[s][nt][0] = fmaf((sacc[0][nt][0] + sacc[1][nt][0]) + (sacc[0][nt][1] + sacc[1][nt][1]),
                            n0 * post[nt], y[s][nt][0]);
-        y[s][nt][1] = fmaf(((sacc2[0][nt][0] + sacc2[1][nt][0]) + (sacc2[0][nt][1] + sacc2[1][nt][1])) +
-                               ((sacc2[0][nt][2] + sacc2[1][nt][2]) + (sacc2[0][nt][3] + sacc2[1][nt][3])),
+        y[s][nt][1] = fmaf((sacc[0][nt][2] + sacc[1][nt][2]) + (sacc[0][nt][3] + sacc[1][nt][3]),
                            n1 * post[nt], y[s][nt][1]);
       }
     }
