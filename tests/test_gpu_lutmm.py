@@ -47,8 +47,10 @@ def test_weight_codes_bit_exact(d, bits, rows):
 
 
 @pytest.mark.parametrize("d,bits", [(128, 3), (128, 4), (64, 3), (256, 2)])
+# m picks the column groups: 4 inputs per CTA up to 4, 8 up to 8, then 16
+# (m = 9 and 16: one group of 16; m = 17: two, the second with one input)
 @pytest.mark.parametrize("rows,k,m", [(80, 512, 1), (64, 1024, 3), (208, 256, 9), (4096, 4096, 1),
-                                      (16, 2048, 5)])
+                                      (16, 2048, 5), (208, 512, 16), (80, 1024, 17)])
 def test_matmul_matches_oracle(d, bits, rows, k, m):
     if k % d:
         pytest.skip("k is not a multiple of head_dim")

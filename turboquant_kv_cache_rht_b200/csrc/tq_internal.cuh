@@ -62,7 +62,7 @@ cudaError_t launch_weights_quantize(const Tables& tb, const void* w, int dtype, 
 // rotated inputs (B-fragment order, with their scales) and, when the plan
 // splits the blocks, the per-split partial sums.
 struct MatmulPlan {
-  int inputs_per_group;  // inputs per CTA column group (4 or 8)
+  int inputs_per_group;  // inputs per CTA column group (4, 8 or 16)
   int groups;            // column groups
   int splits;            // CTAs along the k blocks
   int blocks_per_split;

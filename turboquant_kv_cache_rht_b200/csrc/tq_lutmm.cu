@@ -13,7 +13,7 @@
 // Two kernels.  The first rotates every input block once (one warp per block,
 // warp shuffles), scales it by a power of two that keeps its fp16 hi / lo
 // parts normal, and writes it in the order of the tensor-core B fragments.
-// The second takes 128 weight rows and 4 or 8 inputs per CTA; per block it
+// The second takes 128 weight rows and 4, 8 or 16 inputs per CTA; per block it
 // stages the rows' codes, their norms and the block's input fragments with
 // one 3-stage cp.async pipeline, and each warp scores 2 slabs of 16 rows with
 // a pair table as the decode's keys use (two codes -> an fp16 pair of
@@ -334,6 +334,7 @@ template <int D>
 cudaError_t launch_mm_dim(const Tables& tb, const uint8_t* codes, const uint16_t* norms, int rows,
                           int k, const void* x, int dtype, int m, uint32_t* frag, float* scale,
                           float* partials, float* y, cudaStream_t stream) {
+  if (m > 8) return launch_mm_bits<D, 4>(tb, codes, norms, rows, k, x, dtype, m, frag, scale, partials, y, stream);
   if (m > 4) return launch_mm_bits<D, 2>(tb, codes, norms, rows, k, x, dtype, m, frag, scale, partials, y, stream);
   return launch_mm_bits<D, 1>(tb, codes, norms, rows, k, x, dtype, m, frag, scale, partials, y, stream);
 }
@@ -342,7 +343,7 @@ cudaError_t launch_mm_dim(const Tables& tb, const uint8_t* codes, const uint16_t
 
 MatmulPlan plan_lut_matmul(int rows, int k, int m, int d, long target_ctas) {
   MatmulPlan p;
-  p.inputs_per_group = m > 4 ? 8 : 4;
+  p.inputs_per_group = m > 8 ? 16 : m > 4 ? 8 : 4;
   p.groups = (m + p.inputs_per_group - 1) / p.inputs_per_group;
   const long tiles = std::max<long>(1, (long)((rows + kMmRows - 1) / kMmRows) * p.groups);
   const long nblocks = std::max(1, k / d);
