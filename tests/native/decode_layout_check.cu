@@ -4,6 +4,7 @@
 // warp issues at once fall on distinct banks where the layout promises it.
 // Built and run by tests/test_decode_layout.py; prints "bad N" per shape.
 #include "tq_decode_impl.cuh"
+#include "tq_lutmm.cu"
 
 #include <cstdio>
 #include <set>
@@ -117,7 +118,44 @@ void check_interleaved() {
               Geo::total, g_bad - before);
 }
 
+// LUT matmul, 4-bit codes at d <= 128: table entries 256 bytes apart, the
+// stages' code rows in the entries' second halves
+template <int D, int NT>
+void check_lut() {
+  using Geo = MmGeom<D, 4, NT>;
+  static_assert(Geo::BP, "byte-permute layout");
+  const int before = g_bad;
+  for (int e = 0; e < 256; ++e) CHECK(Geo::offLK + (e << Geo::KSH) == 256 * e);
+  std::set<int> seen;
+  for (int s = 0; s < kMmStages; ++s)
+    for (int r = 0; r < kMmRows; ++r) {
+      for (int w = 0; w < Geo::KS; ++w) {
+        const int p = Geo::code_off(s, r * Geo::KS * 4 + 4 * w);
+        CHECK((p & 255) >= 128 && p + 4 <= 65536);
+        CHECK(seen.insert(p).second);
+        CHECK(p == Geo::code_off(s, r * Geo::KS * 4) + 4 * w);  // a row never straddles two blocks
+      }
+      if (r + 8 < kMmRows)  // the kernel's row g + 8: 2 * 8 * KS words further
+        CHECK(Geo::code_off(s, (r + 8) * Geo::KS * 4) == Geo::code_off(s, r * Geo::KS * 4) + 2 * 8 * Geo::KS * 4);
+    }
+  // a quarter-warp's 16-byte code reads (rows r0 + g, words 4 q .. 4 q + 3) cover 32 banks
+  for (int r0 = 0; r0 < kMmRows; r0 += 16)
+    for (int quarter = 0; quarter < 4; ++quarter) {
+      std::set<int> banks;
+      for (int lane = 8 * quarter; lane < 8 * quarter + 8; ++lane) {
+        const int g = lane >> 2, q = lane & 3;
+        const int p = Geo::code_off(0, (r0 + g) * Geo::KS * 4) + 16 * (q % (Geo::KS / 4));
+        for (int k = 0; k < 4; ++k) banks.insert((p / 4 + k) % 32);
+      }
+      if (Geo::KS == 16) CHECK(banks.size() == 32);
+    }
+  CHECK(Geo::pBase == 65536 && Geo::total == Geo::pBase + kMmStages * Geo::stageA);
+  std::printf("lut d%d nt%d total %d bad %d\n", D, NT, Geo::total, g_bad - before);
+}
+
 int main() {
+  check_lut<128, 1>();
+  check_lut<64, 1>();
   check_pv<1, false>();
   check_pv<4, false>();
   check_pv<8, false>();

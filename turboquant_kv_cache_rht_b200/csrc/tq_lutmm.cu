@@ -48,15 +48,35 @@ struct MmGeom {
   static constexpr int KNW = (QB % 32 == 0) ? QB / 32 : (QB + 16 + 31) / 32;
   static constexpr int LK = 1 << (2 * KB);
   static constexpr int RKL = 5;        // 32 copies: a warp's lookups never share a bank
-  static constexpr int KSH = 2 + RKL;  // 4-byte entries
+  // 4-bit codes at head_dim <= 128, up to 4 inputs (BP): a pair is a whole byte, so with the
+  // table's entries 256 bytes apart one byte permute forms the index (the code
+  // byte above the lane's copy offset).  The other 128 bytes of every entry
+  // form a logical space -- logical x at byte 128 + x + (x & ~127), which keeps
+  // the bank of a plain layout -- holding the stages' code rows (64 or 32
+  // bytes, so no row straddles two blocks); the rest of a stage follows the
+  // 64 KB table region.  Otherwise entries are 128 bytes apart after the stages.
+  // (measured: one input 31.3 -> 30.2 us; with 8 or 16 inputs the larger
+  // stages cost a CTA per SM or more than the indices save, so not there)
+  static constexpr bool BP = KB == 4 && D <= 128 && NT == 1;
+  static constexpr int KSH = BP ? 8 : 2 + RKL;
   static constexpr int FW = frag_words<D, NT>();
-  // one stage: codes [kMmRows][KS], norms [kMmRows], fragments [FW], scales [4 NT]
-  static constexpr int offN = kMmRows * KS * 4;
+  static constexpr int codeBytes = kMmRows * KS * 4;  // code rows of one stage
+  // one stage: codes [kMmRows][KS] (BP: in the logical space), norms
+  // [kMmRows], fragments [FW], scales [4 NT]
+  static constexpr int offN = BP ? 0 : codeBytes;
   static constexpr int offF = offN + kMmRows * 2;
   static constexpr int offS = offF + FW * 4;
   static constexpr int stageA = (offS + 16 * NT + 127) / 128 * 128;
-  static constexpr int offLK = kMmStages * stageA;
-  static constexpr int total = offLK + (LK << KSH);
+  static constexpr int offLK = BP ? 0 : kMmStages * stageA;
+  static constexpr int pBase = BP ? (LK << KSH) : 0;  // stage parts outside the logical space
+  static constexpr int total = BP ? pBase + kMmStages * stageA : offLK + (LK << KSH);
+  // byte of offset x into stage s's code rows
+  __host__ __device__ static constexpr int code_off(int s, int x) {
+    return BP ? 128 + (s * codeBytes + x) + ((s * codeBytes + x) & ~127) : s * stageA + x;
+  }
+  static_assert(!BP || ((KS * 4) % 32 == 0 && 128 % (KS * 4) == 0 && kMmStages * codeBytes <= 32768 &&
+                        codeBytes % 128 == 0),
+                "code rows inside the logical space");
 };
 
 // Input rotation: one warp per (input, block).  frag[(j * groups + cg) * FW ..]
@@ -147,13 +167,14 @@ __global__ void __launch_bounds__(kMmThreads)
   constexpr int NK = (kMmRows * CK + kMmThreads - 1) / kMmThreads;
   constexpr int NF = Geo::FW / 4;  // 16-byte chunks of the fragments
   auto issue_block = [&](int stage, int j) {
-    uint8_t* st = smem + stage * Geo::stageA;
+    uint8_t* st = smem + Geo::pBase + stage * Geo::stageA;
     const uint8_t* src = codes + ((size_t)j * rows + row0) * Geo::kRowB;
 #pragma unroll
     for (int i = 0; i < NK; ++i) {
       const int c = tid + kMmThreads * i, r = c / CK, col = c - r * CK;
       if (c < kMmRows * CK && r < valid_rows)
-        cp_async_chunk<Geo::CBK>(st + r * Geo::KS * 4 + col * Geo::CBK, src + r * Geo::kRowB + col * Geo::CBK);
+        cp_async_chunk<Geo::CBK>(smem + Geo::code_off(stage, r * Geo::KS * 4 + col * Geo::CBK),
+                                 src + r * Geo::kRowB + col * Geo::CBK);
     }
     for (int c = tid; c < valid_rows / 8; c += kMmThreads)  // norms: 16 bytes per 8 rows
       cp_async16(st + Geo::offN + c * 16,
@@ -183,7 +204,8 @@ __global__ void __launch_bounds__(kMmThreads)
     __syncthreads();
     if (it + 2 < nb) issue_block((it + 2) % kMmStages, j0 + it + 2);
     cp_async_commit();
-    const uint8_t* st = smem + (it % kMmStages) * Geo::stageA;
+    const int sidx = it % kMmStages;
+    const uint8_t* st = smem + Geo::pBase + sidx * Geo::stageA;  // norms, fragments, scales
 
     uint32_t bk[NT][Geo::KBLK][2];
     float post[NT];
@@ -215,16 +237,31 @@ __global__ void __launch_bounds__(kMmThreads)
 #pragma unroll
           for (int e = 0; e < 4; ++e) sacc[par][nt][e] = 0.f;
       uint32_t kw0[Geo::KW], kw1[Geo::KW];
-      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(st) + (r0 + g) * Geo::KS;
+      // rows r0 + g and r0 + g + 8 (BP: 8 rows are whole 128-byte blocks apart)
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(smem + Geo::code_off(sidx, (r0 + g) * Geo::KS * 4));
+      const uint32_t* k1 = Geo::BP ? k0 + 2 * 8 * Geo::KS : k0 + 8 * Geo::KS;
+      static_assert(!Geo::BP || (8 * Geo::KS * 4) % 128 == 0, "rows g and g + 8 whole blocks apart");
       load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0, qd, kw0);
-      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k0 + 8 * Geo::KS, qd, kw1);
+      load_value_chunk<Geo::QB, Geo::KW, Geo::KNW>(k1, qd, kw1);
 #pragma unroll
       for (int kb = 0; kb < Geo::KBLK; ++kb) {
         const int o1 = KB * 4 * kb, o2 = o1 + 2 * KB;
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + (field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane));
+        uint32_t i0, i1, i2, i3;
+        if constexpr (Geo::BP) {  // whole code bytes
+          i0 = quad_index<true, 8>(kw0[o1 >> 5], (o1 & 31) >> 3, k_lane);
+          i1 = quad_index<true, 8>(kw1[o1 >> 5], (o1 & 31) >> 3, k_lane);
+          i2 = quad_index<true, 8>(kw0[o2 >> 5], (o2 & 31) >> 3, k_lane);
+          i3 = quad_index<true, 8>(kw1[o2 >> 5], (o2 & 31) >> 3, k_lane);
+        } else {
+          i0 = field_scaled(kw0, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
+          i1 = field_scaled(kw1, Geo::KW, o1, 2 * KB, Geo::KSH) | k_lane;
+          i2 = field_scaled(kw0, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
+          i3 = field_scaled(kw1, Geo::KW, o2, 2 * KB, Geo::KSH) | k_lane;
+        }
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lutK + i0);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lutK + i1);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lutK + i2);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lutK + i3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma16816(sacc[kb & 1][nt], a0, a1, a2, a3, bk[nt][kb][0], bk[nt][kb][1]);
       }
