@@ -127,7 +127,7 @@ void check_lut() {
   const int before = g_bad;
   for (int e = 0; e < 256; ++e) CHECK(Geo::offLK + (e << Geo::KSH) == 256 * e);
   std::set<int> seen;
-  for (int s = 0; s < kMmStages; ++s)
+  for (int s = 0; s < Geo::STG; ++s)
     for (int r = 0; r < kMmRows; ++r) {
       for (int w = 0; w < Geo::KS; ++w) {
         const int p = Geo::code_off(s, r * Geo::KS * 4 + 4 * w);
@@ -149,7 +149,7 @@ void check_lut() {
       }
       if (Geo::KS == 16) CHECK(banks.size() == 32);
     }
-  CHECK(Geo::pBase == 65536 && Geo::total == Geo::pBase + kMmStages * Geo::stageA);
+  CHECK(Geo::pBase == 65536 && Geo::total == Geo::pBase + Geo::STG * Geo::stageA);
   std::printf("lut d%d nt%d total %d bad %d\n", D, NT, Geo::total, g_bad - before);
 }
 

@@ -30,7 +30,10 @@ namespace {
 constexpr int kMmThreads = 128;   // 4 warps
 constexpr int kMmSlabs = 2;       // 16-row slabs per warp
 constexpr int kMmRows = 4 * kMmSlabs * 16;  // weight rows per CTA
-constexpr int kMmStages = 3;
+// pipeline stages: 3, or 2 with 16 inputs per CTA (their fragments double the
+// stage; two stages keep three CTAs per SM)
+template <int NT>
+constexpr int mm_stages() { return NT == 4 ? 2 : 3; }
 constexpr long kMmMaxCtas = kLutMatmulMaxCtas;  // bounds every plan (and so the workspace)
 
 // fragments of one (block, column group): [nt][kb][lane] x 2 words
@@ -67,14 +70,15 @@ struct MmGeom {
   static constexpr int offF = offN + kMmRows * 2;
   static constexpr int offS = offF + FW * 4;
   static constexpr int stageA = (offS + 16 * NT + 127) / 128 * 128;
-  static constexpr int offLK = BP ? 0 : kMmStages * stageA;
+  static constexpr int STG = mm_stages<NT>();
+  static constexpr int offLK = BP ? 0 : STG * stageA;
   static constexpr int pBase = BP ? (LK << KSH) : 0;  // stage parts outside the logical space
-  static constexpr int total = BP ? pBase + kMmStages * stageA : offLK + (LK << KSH);
+  static constexpr int total = BP ? pBase + STG * stageA : offLK + (LK << KSH);
   // byte of offset x into stage s's code rows
   __host__ __device__ static constexpr int code_off(int s, int x) {
     return BP ? 128 + (s * codeBytes + x) + ((s * codeBytes + x) & ~127) : s * stageA + x;
   }
-  static_assert(!BP || ((KS * 4) % 32 == 0 && 128 % (KS * 4) == 0 && kMmStages * codeBytes <= 32768 &&
+  static_assert(!BP || ((KS * 4) % 32 == 0 && 128 % (KS * 4) == 0 && STG * codeBytes <= 32768 &&
                         codeBytes % 128 == 0),
                 "code rows inside the logical space");
 };
@@ -185,10 +189,13 @@ __global__ void __launch_bounds__(kMmThreads)
   };
 
   const int nb = max(0, j1 - j0);
-  if (nb > 0) issue_block(0, j0);
+  constexpr int STG = Geo::STG;
+  if (nb > 0) issue_block(0, j0);  // the first STG - 1 blocks, one commit group each
   cp_async_commit();
-  if (nb > 1) issue_block(1, j0 + 1);
-  cp_async_commit();
+  if constexpr (STG == 3) {
+    if (nb > 1) issue_block(1, j0 + 1);
+    cp_async_commit();
+  }
 
   const uint8_t* lutK = smem + Geo::offLK;
   const uint32_t k_lane = (uint32_t)lane << 2;
@@ -200,11 +207,11 @@ __global__ void __launch_bounds__(kMmThreads)
     for (int nt = 0; nt < NT; ++nt) y[s][nt][0] = y[s][nt][1] = 0.f;
 
   for (int it = 0; it < nb; ++it) {
-    cp_async_wait<1>();
-    __syncthreads();
-    if (it + 2 < nb) issue_block((it + 2) % kMmStages, j0 + it + 2);
+    cp_async_wait<STG - 2>();  // block it has landed
+    __syncthreads();           // and the stage refilled next is no longer read
+    if (it + STG - 1 < nb) issue_block((it + STG - 1) % STG, j0 + it + STG - 1);
     cp_async_commit();
-    const int sidx = it % kMmStages;
+    const int sidx = it % STG;
     const uint8_t* st = smem + Geo::pBase + sidx * Geo::stageA;  // norms, fragments, scales
 
     uint32_t bk[NT][Geo::KBLK][2];
