@@ -46,7 +46,7 @@ def test_weight_codes_bit_exact(d, bits, rows):
     assert np.array_equal(qw.norms.cpu().numpy().view(np.uint16), enc["norm16"].view(np.uint16))
 
 
-@pytest.mark.parametrize("d,bits", [(128, 3), (128, 4), (64, 3), (256, 2)])
+@pytest.mark.parametrize("d,bits", [(128, 3), (128, 4), (64, 3), (64, 4), (256, 2), (256, 4)])
 # m picks the column groups: 4 inputs per CTA up to 4, 8 up to 8, then 16
 # (m = 9 and 16: one group of 16; m = 17: two, the second with one input)
 @pytest.mark.parametrize("rows,k,m", [(80, 512, 1), (64, 1024, 3), (208, 256, 9), (4096, 4096, 1),
