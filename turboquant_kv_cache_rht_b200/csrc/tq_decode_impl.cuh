@@ -592,78 +592,73 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, KB, VB, QJL
   int b = 0, kvh = 0, t_begin = 0, t_end = 0;
   long row_slot = 0;
 
-  // This thread's share of every tile copy: the chunk offsets are the same for
-  // all tiles, so they are computed once (stage offset and tile base vary).
+  // This warp's share of every tile copy: the rows of its own slab, rows
+  // [16 warp, 16 warp + 16) of every array, so that a warp waits for its own
+  // copies only and the tile loop needs no CTA-wide barrier.  The chunk
+  // offsets are the same for all tiles, so they are computed once (stage
+  // offset and tile base vary).
+  constexpr int WR = 16;  // rows per warp
   constexpr int CK = Geo::kRowB / Geo::CBK, CV = Geo::vRowB / Geo::CBV;
-  constexpr int SCH = kDecTile * Geo::sRowB / 16;  // 16-byte chunks of a tile's sign rows (unpadded)
-  constexpr int NK = (kDecTile * CK + kDecThreads - 1) / kDecThreads;
-  constexpr int NV = (kDecTile * CV + kDecThreads - 1) / kDecThreads;
-  constexpr int NS = QJL ? (SCH + kDecThreads - 1) / kDecThreads : 0;
-  int k_dst[NK], k_src[NK], k_row[NK], v_dst[NV], v_src[NV], v_row[NV];
-  int s_dst[NS > 0 ? NS : 1], s_row[NS > 0 ? NS : 1];
+  constexpr int SCH = WR * Geo::sRowB / 16;  // 16-byte chunks of the warp's sign rows
+  constexpr int NK = (WR * CK + 31) / 32;
+  constexpr int NV = (WR * CV + 31) / 32;
+  constexpr int NS = QJL ? (SCH + 31) / 32 : 0;
+  static_assert((WR * Geo::sRowB) % 16 == 0 && (WR * 2) % 16 == 0 && (WR * Geo::MB) % 16 == 0,
+                "a warp's rows of every array are whole 16-byte chunks");
+  int k_dst[NK], k_src[NK], v_dst[NV], v_src[NV];
+  bool k_on[NK], v_on[NV];
 #pragma unroll
   for (int i = 0; i < NK; ++i) {
-    const int c = tid + kDecThreads * i, r = c / CK, col = c - r * CK;
-    k_row[i] = c < kDecTile * CK ? r : kDecTile;
+    const int c = lane + 32 * i, rr = c / CK, col = c - rr * CK, r = WR * warp + rr;
+    k_on[i] = c < WR * CK;
     k_dst[i] = Geo::kvmap(Geo::offK + r * Geo::KS * 4 + col * Geo::CBK);
     k_src[i] = r * Geo::kRowB + col * Geo::CBK;
   }
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
-    const int c = tid + kDecThreads * i, r = c / CV, col = c - r * CV;
-    v_row[i] = c < kDecTile * CV ? r : kDecTile;
+    const int c = lane + 32 * i, rr = c / CV, col = c - rr * CV, r = WR * warp + rr;
+    v_on[i] = c < WR * CV;
     v_dst[i] = Geo::kvmap(Geo::v_row_off(r, col * Geo::CBV / 4));
     v_src[i] = r * Geo::vRowB + col * Geo::CBV;
   }
-#pragma unroll
-  for (int i = 0; i < NS; ++i) {
-    const int c = tid + kDecThreads * i;
-    s_row[i] = c < SCH ? c * 16 / Geo::sRowB : kDecTile;  // first row the chunk holds
-    s_dst[i] = Geo::offS + c * 16;
-  }
   auto issue_tile = [&](int stage, int start) {
+    // nothing when this warp's slab of the tile is empty; otherwise its 16
+    // rows (within capacity: a multiple of 16 past the slab's first token)
+    if (WR * warp >= t_end - start) return;
     uint8_t* skv = smem + Geo::kvBase + stage * Geo::kvStride;  // key and value rows
     uint8_t* st = smem + Geo::pBase + stage * Geo::stageA;       // sign rows and norms
-    const int n_valid = min(kDecTile, t_end - start);
-    const int rows = (n_valid + 15) & ~15;  // within capacity (a multiple of 16)
     const uint8_t* kb = cv.k_codes + (row_slot + start) * Geo::kRowB;
     const uint8_t* vb = cv.v_codes + (row_slot + start) * Geo::vRowB;
 #pragma unroll
     for (int i = 0; i < NK; ++i)
-      if (k_row[i] < rows) cp_async_chunk<Geo::CBK>(skv + k_dst[i], kb + k_src[i]);
+      if (k_on[i]) cp_async_chunk<Geo::CBK>(skv + k_dst[i], kb + k_src[i]);
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-      if (v_row[i] < rows) cp_async_chunk<Geo::CBV>(skv + v_dst[i], vb + v_src[i]);
+      if (v_on[i]) cp_async_chunk<Geo::CBV>(skv + v_dst[i], vb + v_src[i]);
+    const long t0w = row_slot + start + WR * warp;  // the warp's first token
     if constexpr (QJL) {
-      const uint8_t* sb = cv.k_signs + (row_slot + start) * Geo::sRowB;
+      const uint8_t* sb = cv.k_signs + t0w * Geo::sRowB;
+      uint8_t* sd = st + Geo::offS + WR * warp * Geo::sRowB;
 #pragma unroll
-      for (int i = 0; i < NS; ++i)
-        if (s_row[i] < rows) cp_async16(st + s_dst[i], sb + (s_dst[i] - Geo::offS));
-    }
-    if constexpr (AFF) {
-      // (scale, bias) words: rows * NG per array, rows * NG / 4 chunks of 16 bytes
-      const int nc = rows * Geo::NG / 4;
-      const long mo = (row_slot + start) * (long)Geo::MB;
-      for (int c = tid; c < 2 * nc; c += kDecThreads) {
-        const bool vv = c >= nc;
-        const int cc = vv ? c - nc : c;
-        cp_async16(st + (vv ? Geo::offVN : Geo::offKN) + cc * 16,
-                   reinterpret_cast<const uint8_t*>(vv ? cv.v_norm : cv.k_norm) + mo + cc * 16);
+      for (int i = 0; i < NS; ++i) {
+        const int c = lane + 32 * i;
+        if (c < SCH) cp_async16(sd + c * 16, sb + c * 16);
       }
-      if (QJL && tid < rows / 8)
-        cp_async16(st + Geo::offRN + tid * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + tid * 16);
-    } else {
-      // norms: rows * 2 bytes each = rows / 8 chunks per array
-      constexpr int NC = kDecTile / 8;  // 16-byte chunks of one norm array in a full tile
-      static_assert(3 * NC <= kDecThreads, "one thread per norm chunk");
-      const int c = tid % NC, arr = tid / NC;
-      if (c < rows / 8) {
-        if (arr == 0)
-          cp_async16(st + Geo::offKN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_norm + row_slot + start) + c * 16);
-        else if (arr == 1)
-          cp_async16(st + Geo::offVN + c * 16, reinterpret_cast<const uint8_t*>(cv.v_norm + row_slot + start) + c * 16);
-        else if (QJL && arr == 2)
-          cp_async16(st + Geo::offRN + c * 16, reinterpret_cast<const uint8_t*>(cv.k_rnorm + row_slot + start) + c * 16);
+    }
+    // per-token metadata: WR * MB bytes of each of the key and value arrays
+    // (fp16 norms, or the affine codec's (scale, bias) words), WR * 2 of the
+    // QJL residual norms
+    constexpr int CM = WR * Geo::MB / 16, CR = QJL ? WR * 2 / 16 : 0;
+    for (int c = lane; c < 2 * CM + CR; c += 32) {
+      if (c < 2 * CM) {
+        const bool vv = c >= CM;
+        const int cc = vv ? c - CM : c;
+        cp_async16(st + (vv ? Geo::offVN : Geo::offKN) + WR * warp * Geo::MB + cc * 16,
+                   reinterpret_cast<const uint8_t*>(vv ? cv.v_norm : cv.k_norm) + t0w * Geo::MB + cc * 16);
+      } else {
+        const int cc = c - 2 * CM;
+        cp_async16(st + Geo::offRN + WR * warp * 2 + cc * 16,
+                   reinterpret_cast<const uint8_t*>(cv.k_rnorm + t0w) + cc * 16);
       }
     }
   };
@@ -864,8 +859,9 @@ __global__ void __launch_bounds__(kDecThreads, decode_min_ctas<D, G, KB, VB, QJL
   };
 
   for (int it = 0; it < n_tiles; ++it) {
-    cp_async_wait<1>();
-    __syncthreads();
+    cp_async_wait<1>();  // this thread's copies of tile it have landed
+    __syncwarp();        // and the warp's (its slab's rows only), and the stage refilled
+                         // next is no longer read by this warp
     if (it + 2 < n_tiles) issue_tile((it + 2) % kDecStages, t_begin + (it + 2) * kDecTile);
     cp_async_commit();
 
