@@ -62,11 +62,11 @@ DECODE_SOURCES = ("tq_internal.cuh", "tq_decode_impl.cuh", "tq_decode.cu", "tq_d
                   "tq_decode_d256.cu", "tq_decode_affine_d64.cu", "tq_decode_affine_d128.cu",
                   "tq_decode_affine_d256.cu")
 DECODE_TRAFFIC: dict[str, tuple[int, str]] = {
-    "gqa": (31446784, "965c3e25f7b549dd"),
-    "qjl": (567361792, "965c3e25f7b549dd"),
-    "long": (353937152, "965c3e25f7b549dd"),
-    "serving": (1101810176, "965c3e25f7b549dd"),
-    "affine": (38479872, "965c3e25f7b549dd"),
+    "gqa": (31446272, "fb0b4675e697c407"),
+    "qjl": (566612992, "fb0b4675e697c407"),
+    "long": (352942080, "fb0b4675e697c407"),
+    "serving": (1102108672, "fb0b4675e697c407"),
+    "affine": (38473728, "fb0b4675e697c407"),
 }
 
 
@@ -99,11 +99,11 @@ def decode_traffic(workload: str):
 # of active cycles, warp instructions per (token, KV head), warps active %.
 # Keyed, like the traffic, to the digest of the decode sources it describes.
 DECODE_PROFILE: dict[str, tuple[dict, str]] = {
-    "affine": ({"issue_active_pct": 37.2, "warp_inst_per_token_head": 32.93, "warps_active_pct": 12.4}, "965c3e25f7b549dd"),
-    "gqa": ({"issue_active_pct": 41.4, "warp_inst_per_token_head": 33.26, "warps_active_pct": 18.0}, "965c3e25f7b549dd"),
-    "long": ({"issue_active_pct": 47.8, "warp_inst_per_token_head": 41.70, "warps_active_pct": 12.2}, "965c3e25f7b549dd"),
-    "qjl": ({"issue_active_pct": 58.5, "warp_inst_per_token_head": 33.08, "warps_active_pct": 17.7}, "965c3e25f7b549dd"),
-    "serving": ({"issue_active_pct": 61.7, "warp_inst_per_token_head": 23.90, "warps_active_pct": 17.5}, "965c3e25f7b549dd"),
+    "affine": ({"issue_active_pct": 38.1, "warp_inst_per_token_head": 32.16, "warps_active_pct": 12.3}, "fb0b4675e697c407"),
+    "gqa": ({"issue_active_pct": 41.4, "warp_inst_per_token_head": 33.09, "warps_active_pct": 17.6}, "fb0b4675e697c407"),
+    "long": ({"issue_active_pct": 55.9, "warp_inst_per_token_head": 41.47, "warps_active_pct": 12.3}, "fb0b4675e697c407"),
+    "qjl": ({"issue_active_pct": 64.3, "warp_inst_per_token_head": 35.04, "warps_active_pct": 17.3}, "fb0b4675e697c407"),
+    "serving": ({"issue_active_pct": 65.2, "warp_inst_per_token_head": 23.64, "warps_active_pct": 17.0}, "fb0b4675e697c407"),
 }
 
 
