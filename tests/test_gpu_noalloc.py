@@ -3,11 +3,12 @@
 Some callers cannot allocate device memory, so they cannot pass the workspace
 tq_decode_attention needs; tq_decode_attention_noalloc uses a static scratch
 array inside the library instead.  This test calls it through the C ABI twice
-in a row, on different inputs, and checks each result against
-tq_decode_attention with a caller workspace, within the decode tolerance the
-other tests use (the two share the same kernels, so the results agree
-exactly in practice).  It also checks the size limit.  It builds its own
-inputs, so it passes alone in a fresh process as well as after other tests.
+in a row, on different inputs, and checks each result against the CPU oracle
+on the same seeded inputs (per row within the decode tolerance) and against
+tq_decode_attention with a caller workspace (the two share the same kernels,
+so they agree exactly in practice).  It also checks the size limit.  It builds
+its own inputs, so it passes alone in a fresh process as well as after other
+tests.
 """
 import ctypes as C
 
@@ -15,20 +16,33 @@ import numpy as np
 import pytest
 import torch
 
-from tests.tq_helpers import assert_rows_close
+from tests.tq_helpers import assert_rows_close, oracle_decode_unit, oracle_encode_unit, oracle_tables
 
 pytestmark = pytest.mark.gpu
 
 tq = pytest.importorskip("turboquant_kv_cache_rht_b200.tq")
 
 
-def _filled_cache(cb, batch, kv_heads, length, capacity, seed):
+def _raw_kv(batch, kv_heads, length, d, seed):
     g = torch.Generator().manual_seed(seed)
-    k = torch.randn(batch, kv_heads, length, cb.head_dim, generator=g).bfloat16().cuda()
-    v = torch.randn(batch, kv_heads, length, cb.head_dim, generator=g).bfloat16().cuda()
-    cache = tq.Cache(cb, batch, kv_heads, capacity, "cuda")
-    tq.tq_quantize_append(cb, cache, k, v)
+    k = torch.randn(batch, kv_heads, length, d, generator=g).bfloat16()
+    v = torch.randn(batch, kv_heads, length, d, generator=g).bfloat16()
+    return k, v
+
+
+def _filled_cache(cb, k, v, capacity):
+    cache = tq.Cache(cb, k.shape[0], k.shape[1], capacity, "cuda")
+    tq.tq_quantize_append(cb, cache, k.cuda(), v.cuda())
     return cache
+
+
+def _oracle(tb, k, v, q, G):
+    out = np.zeros(q.shape, np.float64)
+    for b in range(k.shape[0]):
+        for h in range(k.shape[1]):
+            ek, ev = oracle_encode_unit(tb, k[b, h], v[b, h])
+            out[b, h * G:(h + 1) * G] = oracle_decode_unit(tb, q[b, h * G:(h + 1) * G], ek, ev)
+    return out
 
 
 def _noalloc(cb, cache, q, out, max_ctx):
@@ -46,20 +60,24 @@ def _noalloc(cb, cache, q, out, max_ctx):
     (128, 4, 4, False, "affine"),      # the affine comparison codec
     (256, 2, 2, True, "gaussian"),     # head_dim 256, 2-bit codes
 ])
-def test_noalloc_matches_workspace_entry_point_twice(d, kb, vb, qjl, codebook):
+def test_noalloc_matches_oracle_twice(d, kb, vb, qjl, codebook):
     cb = tq.Codebook(d, kb, vb, qjl=qjl, seed=3, codebook=codebook)
+    tb = oracle_tables(d, kb, vb, qjl, 3, codebook=codebook)
     cases = [(2, 4, 4, 1000, 1024, 11), (1, 8, 2, 3000, 3008, 12)]   # two calls in a row
     for batch, kv_heads, group, length, cap, seed in cases:
         assert tq.tq_decode_workspace_bytes(cb, batch, kv_heads * group, kv_heads, cap) <= (8 << 20)
-        cache = _filled_cache(cb, batch, kv_heads, length, cap, seed)
+        k, v = _raw_kv(batch, kv_heads, length, d, seed)
+        cache = _filled_cache(cb, k, v, cap)
         g = torch.Generator().manual_seed(seed + 100)
-        q = torch.randn(batch, kv_heads * group, d, generator=g).bfloat16().cuda()
+        q = torch.randn(batch, kv_heads * group, d, generator=g).bfloat16()
         out = torch.full((batch, kv_heads * group, d), float("nan"), device="cuda")
-        got = _noalloc(cb, cache, q, out, cap).clone()
-        ref = tq.tq_decode_attention(cb, cache, q, max_ctx=cap)
+        got = _noalloc(cb, cache, q.cuda(), out, cap).clone()
+        ref = tq.tq_decode_attention(cb, cache, q.cuda(), max_ctx=cap)
         torch.cuda.synchronize()
         assert torch.isfinite(got).all()
-        assert_rows_close(got.cpu().numpy().reshape(-1, d), ref.cpu().numpy().reshape(-1, d))
+        got = got.cpu().numpy().reshape(-1, d)
+        assert_rows_close(got, _oracle(tb, k, v, q, group).reshape(-1, d), what="oracle")
+        assert_rows_close(got, ref.cpu().numpy().reshape(-1, d), what="workspace entry point")
 
 
 def test_noalloc_rejects_decodes_larger_than_its_scratch():
