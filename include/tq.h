@@ -26,6 +26,11 @@
  *  - Pointers are plain host or device addresses as stated per argument; the
  *    library never takes ownership of caller memory and never allocates device
  *    memory.  The only object it allocates is the host-side tq_codebook.
+ *    The library checks device pointers for NULL and alignment only: it does
+ *    not ask the driver whether an address is device memory (that would cost
+ *    a runtime call per pointer on every launch), so a host address passed
+ *    where device memory is required reaches the kernels and faults there.
+ *    Callers check placement (the Python binding does, before each call).
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Device work is enqueued on it and the call returns; results are
  *    visible after the caller synchronizes that stream.

@@ -49,3 +49,28 @@ def test_weights_argument_checks():
     cb = tq.Codebook(128, 4, 4)
     with pytest.raises(ValueError):
         tq.QuantizedWeights(cb, torch.zeros(4, 16, 128))                    # not 2-D
+
+
+def test_host_tensors_are_rejected_before_the_library():
+    """The library takes device pointers; the binding refuses host tensors."""
+    cb = tq.Codebook(128, 3, 4)
+    c = tq.Cache(cb, 1, 2, 32, device="cpu")
+    k = torch.zeros(1, 2, 4, 128)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tq.tq_quantize_append(cb, c, k, k)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tq.tq_quantize_cache(cb, c, k, k, lengths=torch.full((1,), 4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tq.tq_decode_attention(cb, c, torch.zeros(1, 4, 128))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tq.tq_decode_attention_noalloc(cb, c, torch.zeros(1, 4, 128))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tq.QuantizedWeights(cb, torch.zeros(16, 128))
+
+
+def test_output_buffer_checks():
+    tq._check_out("decode", torch.zeros(2, 4, 128), (2, 4, 128))           # accepted
+    for bad in (torch.zeros(2, 4, 64), torch.zeros(2, 4, 128, dtype=torch.float16),
+                torch.zeros(2, 128, 4).transpose(1, 2)):
+        with pytest.raises(ValueError, match="out must be"):
+            tq._check_out("decode", bad, (2, 4, 128))

@@ -195,6 +195,19 @@ class Cache:
         return sum(t.numel() * t.element_size() for t in ts if t is not None)
 
 
+def _on_device(where: str, device: torch.device, **tensors) -> None:
+    """The library takes device pointers: every tensor handed to it must be a
+    CUDA tensor on the device of the cache (or of the encoded weights)."""
+    for name, t in tensors.items():
+        if t is not None and (not t.is_cuda or t.device != device):
+            raise ValueError(f"{where}: {name} must be a CUDA tensor on {device}, not on {t.device}")
+
+
+def _check_out(where: str, out: torch.Tensor, shape) -> None:
+    if out.dtype != torch.float32 or tuple(out.shape) != tuple(shape) or not out.is_contiguous():
+        raise ValueError(f"{where}: out must be a contiguous float32 tensor of shape {tuple(shape)}")
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype not in _DTYPES:
         raise TypeError(f"unsupported dtype {t.dtype}")
@@ -210,6 +223,7 @@ def tq_quantize_append(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Ten
         raise ValueError("k and v must be contiguous")
     if k.shape[0] != cache.batch or k.shape[1] != cache.kv_heads or k.shape[3] != cb.head_dim:
         raise ValueError(f"k shape {tuple(k.shape)} does not match the cache")
+    _on_device("tq_quantize_append", cache.seq_lens.device, cache=cache.seq_lens, k=k, v=v)
     cs = cache.struct()
     _check(lib.tq_quantize_append(cb.handle, C.byref(cs), k.data_ptr(), v.data_ptr(),
                                   _dtype_code(k), k.shape[2], _stream_ptr(stream)),
@@ -233,6 +247,8 @@ def tq_quantize_cache(cb: Codebook, cache: Cache, k: torch.Tensor, v: torch.Tens
         lengths = torch.full((cache.batch,), T, dtype=torch.int32, device=k.device)
     if lengths.dtype != torch.int32 or lengths.shape != (cache.batch,) or not lengths.is_contiguous():
         raise ValueError("lengths must be a contiguous int32 tensor [batch]")
+    _on_device("tq_quantize_cache", cache.seq_lens.device, cache=cache.seq_lens, k=k, v=v,
+               lengths=lengths)
     cs = cache.struct()
     _check(lib.tq_quantize_cache(cb.handle, C.byref(cs), k.data_ptr(), v.data_ptr(), _dtype_code(k),
                                  k.stride(0), k.stride(1), k.stride(2), lengths.data_ptr(), T,
@@ -251,6 +267,7 @@ class QuantizedWeights:
     def __init__(self, cb: Codebook, w: torch.Tensor, stream=None):
         if w.dim() != 2 or not w.is_contiguous():
             raise ValueError("w must be a contiguous [rows, k] CUDA tensor")
+        _on_device("tq_weights_quantize", w.device, w=w)
         self.cb, (self.rows, self.k) = cb, w.shape
         nb = self.k // cb.head_dim
         self.codes = torch.empty(nb, self.rows, cb.layout.k_code_bytes, dtype=torch.uint8, device=w.device)
@@ -270,6 +287,7 @@ class QuantizedWeights:
         """x [m, k] CUDA tensor -> float32 [m, rows] = x W_hat^T."""
         if x.dim() != 2 or x.shape[1] != self.k or not x.is_contiguous():
             raise ValueError(f"x must be a contiguous [m, {self.k}] tensor")
+        _on_device("tq_lut_matmul", self.codes.device, x=x)
         m = x.shape[0]
         y = torch.empty(m, self.rows, dtype=torch.float32, device=x.device)
         nbytes = tq_lut_matmul_workspace_bytes(self.cb, self.rows, self.k, m)
@@ -294,11 +312,16 @@ def tq_decode_attention(cb: Codebook, cache: Cache, q: torch.Tensor, out: torch.
         raise ValueError("q must be contiguous [batch, q_heads, head_dim]")
     hq = q.shape[1]
     max_ctx = cache.capacity if max_ctx is None else max_ctx
+    _on_device("tq_decode_attention", cache.seq_lens.device, cache=cache.seq_lens, q=q, out=out,
+               workspace=workspace)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _check_out("tq_decode_attention", out, q.shape)
     if workspace is None:   # (the library checks a caller's workspace size itself)
         need = tq_decode_workspace_bytes(cb, cache.batch, hq, cache.kv_heads, max_ctx)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_contiguous():
+        raise ValueError("tq_decode_attention: workspace must be contiguous")
     cs = cache.struct()
     _check(lib.tq_decode_attention(cb.handle, C.byref(cs), q.data_ptr(), _dtype_code(q), hq,
                                    float(softmax_scale), int(max_ctx), out.data_ptr(),
@@ -320,8 +343,11 @@ def tq_decode_attention_noalloc(cb: Codebook, cache: Cache, q: torch.Tensor,
     if q.dim() != 3 or q.shape[0] != cache.batch or q.shape[2] != cb.head_dim or not q.is_contiguous():
         raise ValueError("q must be contiguous [batch, q_heads, head_dim]")
     max_ctx = cache.capacity if max_ctx is None else max_ctx
+    _on_device("tq_decode_attention_noalloc", cache.seq_lens.device, cache=cache.seq_lens, q=q,
+               out=out)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _check_out("tq_decode_attention_noalloc", out, q.shape)
     cs = cache.struct()
     _check(lib.tq_decode_attention_noalloc(cb.handle, C.byref(cs), q.data_ptr(), _dtype_code(q),
                                            q.shape[1], float(softmax_scale), int(max_ctx),
