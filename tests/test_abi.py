@@ -235,3 +235,23 @@ def test_bench_byte_model_matches_the_layout(name):
     per_token = (lay.k_code_bytes + lay.v_code_bytes + 2 * 2 * lay.norm_halves
                  + ((lay.k_sign_bytes + 2) if w.qjl else 0))
     assert bench.token_bytes(w) == per_token
+    # and the arrays a cache allocates from that layout hold exactly that much
+    cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, codebook=w.codebook)
+    assert tq.Cache(cb, 2, 3, 32, device="cpu").nbytes() == 2 * 3 * 32 * per_token
+
+
+def test_bench_step_bytes():
+    """3.5 bits at d 128 reads 48 + 64 + 4 bytes per (token, KV head), 4.41x
+    fewer than bf16; a step's decode bytes are the rows' cache bytes plus the
+    bf16 queries read and fp32 outputs written, its append one K and one V
+    vector in and out per (row, KV head)."""
+    import bench
+    from turboquant_kv_cache_rht_b200 import workloads as wl
+    assert bench.token_bytes(wl.WORKLOADS["serving"]) == 116
+    w = wl.with_sizes(wl.WORKLOADS["gqa"], context=100, batch=3)
+    lens = [100, 37, 0]
+    sb = bench.step_bytes(w, lens)
+    d = w.head_dim
+    assert sb["decode"] == sum(lens) * w.kv_heads * 116 + w.batch * w.q_heads * d * (2 + 4)
+    assert sb["append"] == w.batch * w.kv_heads * (2 * d * 2 + (3 + 4) * d // 8 + 4)
+    assert sb["total"] == sb["decode"] + sb["append"]
