@@ -20,7 +20,10 @@ read by the decode, queries, outputs, appended K/V and their codes) / device
 time, in GB/s, plus ctx-tokens/s, the decode call's roofline against the
 measured HBM copy bandwidth, bulk quantize Mvec/s, an end-to-end figure through
 host buffers, the FP16/BF16 dense decode baselines on the same GPU, and the CPU
-oracle timed on the host as a baseline.  The default workload is `serving`
+oracle timed on the host as a baseline.  That oracle leg also checks the
+benchmark's own inputs: the unit it encodes and decodes goes through the
+library too, and `cpu_baseline.parity` reports the largest per-row error of
+the GPU output against the oracle's (bar: 2e-3 of the row's largest value).  The default workload is `serving`
 (32 ragged rows of 8k-64k tokens); the line also carries `long_context`: the
 decode calls of the 131k-token `qjl` and 524k-token `long` workloads with their
 own roofline fractions and dense baselines.  `roofline.traffic` (ncu DRAM
@@ -707,9 +710,43 @@ class OracleUnit:
         return (self.T + 1) * token_bytes(w) + w.group * d * (esz + 4) + 2 * d * esz + vec_out
 
 
+def unit_parity(u: "OracleUnit", ref) -> dict:
+    """The benchmark's own inputs checked against the oracle: the unit the
+    oracle leg encodes (batch row 0, KV head 0: its whole context, then the
+    first step's appended token) goes through the library on the GPU as well,
+    and each of the G output rows must be within the decode tolerance of the
+    oracle's (max |gpu - oracle| <= 2e-3 * max |oracle| per row).  A failure
+    is reported in the line and on stderr; it does not stop the benchmark."""
+    import numpy as np
+    from turboquant_kv_cache_rht_b200 import tq
+    w = u.w
+    try:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        cb = tq.Codebook(w.head_dim, w.k_bits, w.v_bits, w.qjl, w.rht_seed, codebook=w.codebook)
+        cache = tq.Cache(cb, 1, 1, (u.T + 1 + 15) // 16 * 16, dev)
+        k, v = wl.kv_unit(w, 0, 0, u.T)
+        tq.tq_quantize_cache(cb, cache, k[None, None].to(dev), v[None, None].to(dev))
+        kn, vn = wl.kv_step(w, 0)
+        tq.tq_quantize_append(cb, cache, kn[0:1, 0:1].contiguous().to(dev),
+                              vn[0:1, 0:1].contiguous().to(dev))
+        q = wl.queries(w, 0)[0:1, :w.group].contiguous().to(dev)
+        got = tq.tq_decode_attention(cb, cache, q)[0].double().cpu().numpy()
+        status = int(cache.status.item())
+        ref = np.asarray(ref, np.float64)
+        err = max(float(np.abs(got[r] - ref[r]).max() / np.abs(ref[r]).max()) for r in range(ref.shape[0]))
+        res = {"unit": "batch row 0, KV head 0", "tokens": u.T + 1, "rows": int(ref.shape[0]),
+               "max_rel_err": float(f"{err:.3g}"), "tol": 2e-3, "status": status,
+               "ok": bool(err <= 2e-3 and status == 0)}
+    except Exception as e:  # the check must not cost the measurement
+        res = {"error": f"{type(e).__name__}: {e}", "ok": False}
+    if not res["ok"]:
+        print(f"bench: parity check against the oracle failed: {res}", file=sys.stderr, flush=True)
+    return res
+
+
 def cpu_baseline(w: wl.Workload, budget_s: float = 10.0) -> dict:
     u = OracleUnit(w)
-    u.step()
+    parity = unit_parity(u, u.step())
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -724,6 +761,7 @@ def cpu_baseline(w: wl.Workload, budget_s: float = 10.0) -> dict:
                      f"decode {w.group} query heads over {u.T + 1} tokens (numpy, float64 attention)",
            "host_cpus": os.cpu_count()}
     res.update(oracle_rates(u))
+    res["parity"] = parity
     return res
 
 
