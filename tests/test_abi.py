@@ -74,6 +74,13 @@ def test_codebook_rejects_bad_params(bad):
     assert tq.tq_last_error()
 
 
+def test_codebook_init_null_arguments():
+    params = tq.tq_params(128, 3, 4, 0, 0, 0)
+    h = C.c_void_p()
+    assert tq.lib.tq_codebook_init(None, C.byref(h), None) == tq.TQ_ERR_INVALID
+    assert tq.lib.tq_codebook_init(C.byref(params), None, None) == tq.TQ_ERR_INVALID
+
+
 def test_affine_layout_matches_the_pages_memory_table(golden):
     """The library's per-vector bytes for the affine codec reproduce the
     "Memory footprint over long context" KB/token figures (the fp16 row fixes
@@ -128,8 +135,15 @@ def test_append_validation():
     assert _append(cb, _fake_cache(), k=0) == tq.TQ_ERR_INVALID
     assert _append(cb, _fake_cache(), k=(1 << 12) + 4) == tq.TQ_ERR_INVALID
     assert _append(cb, _fake_cache(), n_new=0) == tq.TQ_OK                 # no-op, no launch
+    assert _append(cb, _fake_cache(), n_new=65) == tq.TQ_ERR_INVALID       # past the capacity
+    assert "exceeds capacity" in tq.tq_last_error()
+    big = dict(batch=1 << 30, kv_heads=1 << 30, capacity=1 << 30)           # sizes only
+    assert _append(cb, _fake_cache(**big)) == tq.TQ_ERR_INVALID
+    assert "too large" in tq.tq_last_error()
     qcb = tq.Codebook(128, 3, 4, qjl=True)
     assert _append(qcb, _fake_cache()) == tq.TQ_ERR_INVALID                # QJL needs k_signs
+    assert _append(qcb, _fake_cache(qjl=True, k_rnorm=(1 << 21) + 2)) == tq.TQ_ERR_INVALID
+    assert "not 16-byte aligned" in tq.tq_last_error()
     assert tq.lib.tq_quantize_append(None, C.byref(_fake_cache()), 1 << 12, 1 << 13, 1, 1,
                                      None) == tq.TQ_ERR_INVALID
 
@@ -172,9 +186,12 @@ def test_weights_validation():
     mm = lambda rows=64, k=512, m=1, ws=0, nbytes=0, y=1 << 15: tq.lib.tq_lut_matmul(
         cb.handle, 1 << 13, 1 << 14, rows, k, 1 << 12, 1, m, y, ws, nbytes, None)
     assert mm(m=0) == tq.TQ_ERR_INVALID
+    assert mm(m=65535 * 4 + 1) == tq.TQ_ERR_INVALID
     assert mm(y=0) == tq.TQ_ERR_INVALID
+    assert mm(y=(1 << 15) + 8) == tq.TQ_ERR_INVALID   # misaligned output
     need = tq.tq_lut_matmul_workspace_bytes(cb, 64, 512, 1)
     assert need > 0 and mm(ws=1 << 16, nbytes=need - 4) == tq.TQ_ERR_CAPACITY
+    assert mm(ws=(1 << 16) + 4, nbytes=need) == tq.TQ_ERR_INVALID       # misaligned workspace
     assert tq.tq_lut_matmul_workspace_bytes(cb, 64, 500, 1) == 0       # bad k
     # rotated inputs: 4 blocks x 1 group of 4 inputs x (8 k-blocks x 32 lanes x 2 words
     # + 4 scales); 64 rows x 1 group is one tile, so the 4 blocks are split one per
@@ -185,9 +202,10 @@ def test_weights_validation():
     assert tq.tq_lut_matmul_workspace_bytes(cb, 128 * 600, 512, 8) == (4 * 2 * 8 * 64 + 4 * 8) * 4
 
 
-def _decode(cb, cache, q_heads=4, max_ctx=64, ws=1 << 14, ws_bytes=1 << 30, scale=0.0, q=1 << 12):
+def _decode(cb, cache, q_heads=4, max_ctx=64, ws=1 << 14, ws_bytes=1 << 30, scale=0.0, q=1 << 12,
+            out=1 << 13):
     return tq.lib.tq_decode_attention(cb.handle, C.byref(cache), q, 1, q_heads, scale, max_ctx,
-                                      1 << 13, ws, ws_bytes, None)
+                                      out, ws, ws_bytes, None)
 
 
 def test_decode_validation():
@@ -196,6 +214,12 @@ def test_decode_validation():
     assert _decode(cb, _fake_cache(), max_ctx=65) == tq.TQ_ERR_INVALID      # past capacity
     assert _decode(cb, _fake_cache(), ws_bytes=16) == tq.TQ_ERR_CAPACITY
     assert _decode(cb, _fake_cache(), q=0) == tq.TQ_ERR_INVALID
+    assert _decode(cb, _fake_cache(), max_ctx=-1) == tq.TQ_ERR_INVALID
+    assert _decode(cb, _fake_cache(), q=(1 << 12) + 2) == tq.TQ_ERR_INVALID     # misaligned q
+    assert _decode(cb, _fake_cache(), out=(1 << 13) + 4) == tq.TQ_ERR_INVALID   # misaligned out
+    assert _decode(cb, _fake_cache(), ws=(1 << 14) + 8) == tq.TQ_ERR_INVALID    # misaligned workspace
+    assert "16-byte aligned" in tq.tq_last_error()
+    assert _decode(cb, _fake_cache(), ws=0) == tq.TQ_ERR_CAPACITY              # no workspace
     assert _decode(cb, _fake_cache(), scale=float("nan")) == tq.TQ_ERR_INVALID
     assert _decode(cb, _fake_cache(kv_heads=1), q_heads=3) == tq.TQ_ERR_UNSUPPORTED   # group 3
     assert _decode(cb, _fake_cache(kv_heads=1), q_heads=16) == tq.TQ_ERR_UNSUPPORTED  # group 16
