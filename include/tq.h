@@ -138,7 +138,8 @@ typedef struct tq_codebook tq_codebook;  /* opaque, host memory, owned by the li
  * Packed code layout of one vector: a little-endian bit stream in which
  * channel i's b-bit code occupies bits [b*i, b*i + b), bit 0 being the least
  * significant bit of byte 0; the sign plane is the same stream with b = 1.
- * capacity must be a multiple of 16.  Every pointer must be 16-byte aligned. */
+ * capacity must be a multiple of 16 and batch at most 65535.  Every pointer
+ * must be 16-byte aligned. */
 typedef struct {
   uint8_t *k_codes, *v_codes, *k_signs;
   uint16_t *k_norm, *v_norm, *k_rnorm;

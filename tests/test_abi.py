@@ -137,7 +137,9 @@ def test_append_validation():
     assert _append(cb, _fake_cache(), n_new=0) == tq.TQ_OK                 # no-op, no launch
     assert _append(cb, _fake_cache(), n_new=65) == tq.TQ_ERR_INVALID       # past the capacity
     assert "exceeds capacity" in tq.tq_last_error()
-    big = dict(batch=1 << 30, kv_heads=1 << 30, capacity=1 << 30)           # sizes only
+    assert _append(cb, _fake_cache(batch=65536)) == tq.TQ_ERR_INVALID      # one grid row per batch row
+    assert "65535" in tq.tq_last_error()
+    big = dict(batch=65535, kv_heads=1 << 30, capacity=1 << 30)             # sizes only
     assert _append(cb, _fake_cache(**big)) == tq.TQ_ERR_INVALID
     assert "too large" in tq.tq_last_error()
     qcb = tq.Codebook(128, 3, 4, qjl=True)
@@ -215,6 +217,7 @@ def test_decode_validation():
     assert _decode(cb, _fake_cache(), ws_bytes=16) == tq.TQ_ERR_CAPACITY
     assert _decode(cb, _fake_cache(), q=0) == tq.TQ_ERR_INVALID
     assert _decode(cb, _fake_cache(), max_ctx=-1) == tq.TQ_ERR_INVALID
+    assert _decode(cb, _fake_cache(batch=70000)) == tq.TQ_ERR_INVALID       # merge grid rows
     assert _decode(cb, _fake_cache(), q=(1 << 12) + 2) == tq.TQ_ERR_INVALID     # misaligned q
     assert _decode(cb, _fake_cache(), out=(1 << 13) + 4) == tq.TQ_ERR_INVALID   # misaligned out
     assert _decode(cb, _fake_cache(), ws=(1 << 14) + 8) == tq.TQ_ERR_INVALID    # misaligned workspace

@@ -272,6 +272,8 @@ tq_status check_cache(const tq_codebook* cb, const tq_cache* c) {
                 c->batch, c->kv_heads, c->capacity);
   if (c->capacity % 16 != 0)
     return fail(TQ_ERR_INVALID, "capacity %d is not a multiple of 16", c->capacity);
+  // the append, conversion and merge grids index batch rows by blockIdx.y
+  if (c->batch > 65535) return fail(TQ_ERR_INVALID, "batch %d: at most 65535 rows", c->batch);
   const void* need[] = {c->k_codes, c->v_codes, c->k_norm, c->v_norm, c->seq_lens, c->status,
                         c->append_sync};
   const char* names[] = {"k_codes", "v_codes", "k_norm", "v_norm", "seq_lens", "status",
