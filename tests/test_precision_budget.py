@@ -1,22 +1,29 @@
-"""What the decode's fp16 code tables cost of the 2e-3 bar (CPU only).
+"""What the decode's fp16 operands cost of the 2e-3 bar (CPU only).
 
 The decode kernel feeds the tensor cores fp16 operands.  Its code tables hold
 fp16(lam * c_j) for the Lloyd-Max levels c_j and a per-codebook scale lam in
 [1, 2), formed as an fp32 product and divided out again in fp32 after the
 accumulation; the scale is the one of a 2^16-step grid whose roundings come
-closest to the exact products.  These checks restate that search and bound,
-with the oracle on the workloads' own inputs, what the rounded tables alone
-change in the decode output, so that the GPU parity bar keeps its margin for
-the other roundings (the fp16 hi + lo query and weights, the accumulation
-order, the hardware exp2):
+closest to the exact products.  The query and the softmax weights enter as
+fp16 hi + lo pairs.  These checks restate that search and bound, with the
+oracle's steps on the workloads' own inputs, what those roundings change in
+the decode output, so that the GPU parity bar keeps its margin for the rest
+(the fp32 accumulation order, the hardware exp2):
 
 * the best scale brings the largest relative rounding error of the 2-, 3- and
   4-bit levels to about 3e-7, 2e-5 and 1e-4, where plain fp16 has 2e-4 to
   3e-4;
 * with the scaled tables the decode stays within 2e-4 of the exact output on
   the gqa, qjl and long inputs, whereas plain fp16 tables alone would use
-  most of the 2e-3 bar on the gqa inputs.
+  most of the 2e-3 bar on the gqa inputs;
+* rounding, in addition, the rotated query (and the QJL query) and the
+  softmax weights times the value norms to fp16 hi + lo pairs under a
+  power-of-two scale, as the kernel's MMA operands are, keeps the output
+  within 2e-4; a single fp16 query instead would cost over 1e-3 on the long
+  inputs.
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -80,3 +87,55 @@ def test_scaled_tables_leave_the_bar_its_margin(name):
     assert plain > 3 * scaled
     if name == "gqa":
         assert plain > 1e-3          # plain fp16 tables alone: over half of the 2e-3 bar
+
+
+def _fp16_operand(x, split=True):
+    """x rounded as an MMA operand row: scaled by a power of two (largest
+    magnitude in [2^7, 2^8)), then fp16 hi, plus fp16 of the remainder."""
+    scale = np.ldexp(1.0, 8 - np.frexp(np.abs(x).max(axis=-1, keepdims=True))[1])
+    xs = x * scale
+    hi = xs.astype(np.float16).astype(np.float64)
+    lo = (xs - hi).astype(np.float16).astype(np.float64) if split else 0.0
+    return (hi + lo) / scale
+
+
+def _operand_rounding_error(name, split_query=True, T=4096):
+    """The oracle's rotated-frame decode with the kernel's operand roundings:
+    scaled fp16 tables, query and weights as fp16 operands."""
+    w = wl.WORKLOADS[name]
+    d = w.head_dim
+    ck, bk = o.codebook(w.k_bits)
+    cv, bv = o.codebook(w.v_bits)
+    s1 = o.rotation_signs(w.rht_seed, d)
+    s2 = o.rotation_signs(w.rht_seed, d, second=True) if w.qjl else None
+    k, v = wl.kv_unit(w, 0, 0, T)
+    ek = o.encode(k.float().numpy(), s1, ck, bk, w.k_bits, s2)
+    ev = o.encode(v.float().numpy(), s1, cv, bv, w.v_bits)
+    q = wl.queries(w, 0)[0, :w.group].float().numpy().astype(np.float64)
+    kw = dict(s2=s2, k_sign_bits=ek["sign_bits"], k_rnorm16=ek["rnorm16"]) if w.qjl else {}
+    exact = o.decode_attention(q, s1, ek["idx"], ek["norm16"], ck, ev["idx"], ev["norm16"], cv, **kw)
+
+    q_rot = o.rht_forward(q, s1)
+    scores = _fp16_operand(q_rot, split_query) @ o.dequantize_rotated(ek["idx"], ek["norm16"],
+                                                                       _scaled_table(ck)).T
+    if w.qjl:
+        q_hat = _fp16_operand(o.rht_forward(q_rot, s2), split_query)
+        signs = 2.0 * ek["sign_bits"] - 1.0
+        scores = scores + (math.sqrt(math.pi / (2 * d)) * ek["rnorm16"].astype(np.float64)[None, :]
+                           * (q_hat @ signs.T))
+    scores = scores / math.sqrt(d)
+    p = np.exp(scores - scores.max(axis=1, keepdims=True))
+    weights = _fp16_operand(p * ev["norm16"].astype(np.float64)[None, :])
+    o_rot = (weights @ _scaled_table(cv)[ev["idx"]]) / p.sum(axis=1, keepdims=True) / math.sqrt(d)
+    out = o.rht_inverse(o_rot, s1)
+    return float((np.abs(out - exact).max(axis=1) / np.abs(exact).max(axis=1)).max())
+
+
+@pytest.mark.parametrize("name", ["gqa", "qjl", "long", "serving"])
+def test_split_operands_keep_the_margin(name):
+    split = _operand_rounding_error(name)
+    single = _operand_rounding_error(name, split_query=False)
+    assert split < 2e-4
+    assert single > 3 * split
+    if name == "long":
+        assert single > 1e-3          # a single fp16 query: over half of the bar at d 256
