@@ -20,7 +20,12 @@ the decode output, so that the GPU parity bar keeps its margin for the rest
   softmax weights times the value norms to fp16 hi + lo pairs under a
   power-of-two scale, as the kernel's MMA operands are, keeps the output
   within 2e-4; a single fp16 query instead would cost over 1e-3 on the long
-  inputs.
+  inputs;
+* the affine comparison codec forms each value operand as scale * level +
+  bias with one fp16 rounding (a fused multiply-add in half precision); that
+  rounding is what its decode error is made of, about 3e-4 (the GPU parity
+  tests measure 2.5e-4 to 3e-4), inside the bar but some 1000 times what the
+  same decode with exact values shows.
 """
 import math
 
@@ -139,3 +144,30 @@ def test_split_operands_keep_the_margin(name):
     assert single > 3 * split
     if name == "long":
         assert single > 1e-3          # a single fp16 query: over half of the bar at d 256
+
+
+def test_affine_value_operands():
+    w = wl.WORKLOADS["affine"]
+    d, T = w.head_dim, 4096
+    s1 = o.rotation_signs(w.rht_seed, d)
+    k, v = wl.kv_unit(w, 0, 0, T)
+    ek = o.affine_encode(k.float().numpy(), w.k_bits, s1)
+    ev = o.affine_encode(v.float().numpy(), w.v_bits)
+    q = wl.queries(w, 0)[0, :w.group].float().numpy().astype(np.float64)
+    exact = o.affine_decode_attention(q, s1, ek, ev)
+
+    keys = o.affine_dequantize(ek["idx"], ek["scale16"], ek["bias16"])
+    scores = _fp16_operand(o.rht_forward(q, s1)) @ keys.T / math.sqrt(d)
+    p = np.exp(scores - scores.max(axis=1, keepdims=True))
+    weights = _fp16_operand(p)
+    n, groups = T, d // 64
+    scale = ev["scale16"].astype(np.float64).reshape(n, groups, 1)
+    bias = ev["bias16"].astype(np.float64).reshape(n, groups, 1)
+    levels = ev["idx"].reshape(n, groups, 64).astype(np.float64)
+    fma16 = (scale * levels + bias).astype(np.float16).astype(np.float64).reshape(n, d)  # one rounding
+    rel = lambda a: float((np.abs(a - exact).max(axis=1) / np.abs(exact).max(axis=1)).max())
+    with_fma = rel((weights @ fma16) / p.sum(axis=1, keepdims=True))
+    exact_values = rel((weights @ o.affine_dequantize(ev["idx"], ev["scale16"], ev["bias16"]))
+                       / p.sum(axis=1, keepdims=True))
+    assert 1e-4 < with_fma < 6e-4
+    assert exact_values < with_fma / 100
