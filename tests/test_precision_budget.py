@@ -25,7 +25,9 @@ the decode output, so that the GPU parity bar keeps its margin for the rest
   bias with one fp16 rounding (a fused multiply-add in half precision); that
   rounding is what its decode error is made of, about 3e-4 (the GPU parity
   tests measure 2.5e-4 to 3e-4), inside the bar but some 1000 times what the
-  same decode with exact values shows.
+  same decode with exact values shows;
+* the weights-regime LUT matmul uses the same scaled tables and split inputs:
+  its product stays within 1.2e-4 of the oracle's for 2-, 3- and 4-bit codes.
 """
 import math
 
@@ -171,3 +173,26 @@ def test_affine_value_operands():
                        / p.sum(axis=1, keepdims=True))
     assert 1e-4 < with_fma < 6e-4
     assert exact_values < with_fma / 100
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_lut_matmul_operands(bits):
+    d, rows, k, m = 128, 256, 1024, 4
+    rng = np.random.default_rng(7 + bits)
+    w = rng.standard_normal((rows, k)).astype(np.float32)
+    x = rng.standard_normal((m, k))
+    levels, bounds = o.codebook(bits)
+    s1 = o.rotation_signs(5, d)
+    enc = o.weights_encode(w, s1, levels, bounds, bits)
+    exact = o.lut_matmul(x, enc["idx"], enc["norm16"], s1, levels)
+
+    def product(table):
+        y = np.zeros((m, rows))
+        for j in range(k // d):   # per block: split rotated input . (n16 * table[code] / sqrt d)
+            xr = _fp16_operand(o.rht_forward(x[:, j * d:(j + 1) * d], s1))
+            y += xr @ o.dequantize_rotated(enc["idx"][j], enc["norm16"][j], table).T
+        return float((np.abs(y - exact).max(axis=1) / np.abs(exact).max(axis=1)).max())
+
+    scaled, plain = product(_scaled_table(levels)), product(_plain_table(levels))
+    assert scaled < 1.2e-4
+    assert plain > 2 * scaled
