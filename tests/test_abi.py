@@ -6,6 +6,8 @@ import re
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle as o
 from turboquant_kv_cache_rht_b200 import tq
@@ -234,15 +236,64 @@ def test_workspace_size_formula():
     # slots (one wave of at most 592 CTAs, no more CTAs than tiles, + units - 1)
     # x group x (head_dim + 2) floats
     def expect(batch, q_heads, kv_heads, max_ctx, d=128):
-        units = batch * kv_heads
-        ctas = max(1, min(148 * 4, units * max(1, -(-max_ctx // 64))))
-        return (ctas + units - 1) * (q_heads // kv_heads) * (d + 2) * 4
+        return _expect_decode_workspace(batch, q_heads, kv_heads, max_ctx, d)
     cb = tq.Codebook(128, 3, 4)
     for args in ((1, 32, 8, 32768), (32, 32, 8, 65536), (1, 1, 1, 100), (1, 1, 1, 0), (4, 8, 8, 64)):
         assert tq.tq_decode_workspace_bytes(cb, *args) == expect(*args), args
     assert tq.tq_decode_workspace_bytes(cb, 1, 30, 8, 100) == 0              # group 3.75
     cb256 = tq.Codebook(256, 2, 2)
     assert tq.tq_decode_workspace_bytes(cb256, 2, 16, 4, 524288) == expect(2, 16, 4, 524288, 256)
+
+
+def _expect_decode_workspace(batch, q_heads, kv_heads, max_ctx, d):
+    units = batch * kv_heads
+    ctas = max(1, min(148 * 4, units * max(1, -(-max_ctx // 64))))
+    return (ctas + units - 1) * (q_heads // kv_heads) * (d + 2) * 4
+
+
+@settings(max_examples=300, deadline=None)
+@given(batch=st.integers(1, 300), kv_heads=st.sampled_from([1, 2, 4, 8, 16]),
+       group=st.sampled_from([1, 2, 4, 8]), max_ctx=st.integers(0, 1 << 21),
+       d=st.sampled_from([64, 128, 256]))
+def test_decode_workspace_formula_random(batch, kv_heads, group, max_ctx, d):
+    cb = _codebook_cache(d)
+    got = tq.tq_decode_workspace_bytes(cb, batch, kv_heads * group, kv_heads, max_ctx)
+    assert got == _expect_decode_workspace(batch, kv_heads * group, kv_heads, max_ctx, d)
+
+
+def _expect_lut_workspace(rows, k, m, d, max_ctas=148 * 4):
+    """The weights-regime plan restated: 128-row tiles times column groups of
+    4, 8 or 16 inputs; the k/d blocks split so that tiles x splits stays within
+    one wave; workspace = rotated inputs + their scales + split partials."""
+    per_group = 16 if m > 8 else 8 if m > 4 else 4
+    groups = -(-m // per_group)
+    tiles = max(1, -(-rows // 128) * groups)
+    nblocks = max(1, k // d)
+    s = max(1, min(nblocks, max_ctas // tiles))
+    per_split = -(-nblocks // s)
+    splits = -(-nblocks // per_split)
+    frag_words = nblocks * groups * (per_group // 4) * (d // 16) * 64
+    scales = nblocks * groups * per_group
+    partials = splits * m * rows if splits > 1 else 0
+    return (frag_words + scales + partials) * 4
+
+
+@settings(max_examples=300, deadline=None)
+@given(rows=st.integers(1, 2048).map(lambda r: 16 * r), blocks=st.integers(1, 96),
+       m=st.integers(1, 64), d=st.sampled_from([64, 128, 256]))
+def test_lut_workspace_formula_random(rows, blocks, m, d):
+    cb = _codebook_cache(d)
+    assert tq.tq_lut_matmul_workspace_bytes(cb, rows, blocks * d, m) == _expect_lut_workspace(
+        rows, blocks * d, m, d)
+
+
+_CODEBOOKS = {}
+
+
+def _codebook_cache(d):
+    if d not in _CODEBOOKS:
+        _CODEBOOKS[d] = tq.Codebook(d, 4, 4)
+    return _CODEBOOKS[d]
 
 
 def test_kv_bits_split_matches_oracle():
