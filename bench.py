@@ -23,7 +23,9 @@ host buffers, the FP16/BF16 dense decode baselines on the same GPU, and the CPU
 oracle timed on the host as a baseline.  That oracle leg also checks the
 benchmark's own inputs: the unit it encodes and decodes goes through the
 library too, and `cpu_baseline.parity` reports the largest per-row error of
-the GPU output against the oracle's (bar: 2e-3 of the row's largest value).  The default workload is `serving`
+the GPU output against the oracle's (bar: 2e-3 of the row's largest value).
+`cpu_baseline.rates_by_workload` gives the oracle's quantize and decode rates
+for every workload, on one thread and on all, each on a bounded sample.  The default workload is `serving`
 (32 ragged rows of 8k-64k tokens); the line also carries `long_context`: the
 decode calls of the 131k-token `qjl` and 524k-token `long` workloads with their
 own roofline fractions and dense baselines.  `roofline.traffic` (ncu DRAM
@@ -761,8 +763,24 @@ def cpu_baseline(w: wl.Workload, budget_s: float = 10.0) -> dict:
                      f"decode {w.group} query heads over {u.T + 1} tokens (numpy, float64 attention)",
            "host_cpus": os.cpu_count()}
     res.update(oracle_rates(u))
+    res["rates_by_workload"] = oracle_rates_by_workload()
     res["parity"] = parity
     return res
+
+
+def oracle_rates_by_workload(context: int = 8192, budget_s: float = 0.3) -> dict:
+    """The oracle's quantize and decode rates (as ``oracle_rates``) for every
+    workload, each on a bounded sample: batch row 0, KV head 0 at `context`
+    tokens (the workload's own context when shorter).  Per-token and
+    per-vector costs do not depend on the context length beyond that."""
+    out = {}
+    for name, w in sorted(wl.WORKLOADS.items()):
+        try:  # a reported baseline: a failure here must not cost the line
+            u = OracleUnit(wl.with_sizes(w, context=min(context, w.context or context)))
+            out[name] = dict(oracle_rates(u, budget_s), sample_tokens=u.T + 1)
+        except Exception as e:
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+    return out
 
 
 def oracle_rates(u: "OracleUnit", budget_s: float = 2.0) -> dict:
@@ -820,7 +838,8 @@ def run_reference(args, rank: int) -> dict | None:
                    "sample": "one (batch row, KV head) unit of the workload per step"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": f"per step: encode 1 appended K and V, decode {w.group} query heads "
-                                   f"over {u.T + 1} tokens of one KV head"},
+                                   f"over {u.T + 1} tokens of one KV head",
+                         "rates_by_workload": oracle_rates_by_workload()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -32,6 +32,11 @@ def test_reference_arm_json_line(workload):
     assert d["config"]["workload"] == workload
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    rates = cb["rates_by_workload"]          # every workload, one thread and all threads
+    assert set(rates) == {"tiny", "gqa", "qjl", "long", "serving", "affine"}
+    for r in rates.values():
+        for mode in ("all_threads", "one_thread"):
+            assert r[mode]["quantize_mvec_s"] > 0 and r[mode]["decode_ctx_tokens_s"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
 
