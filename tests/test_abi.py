@@ -21,6 +21,39 @@ def _declared():
     return sorted(set(re.findall(r"\b(tq_[a-z_0-9]+)\s*\(", src)))
 
 
+def test_plain_c_client(tmp_path):
+    """include/tq.h compiles as strict C99 and a C program linked against
+    libtq.so gets the same answers as the Python binding (host-only calls)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.dirname(os.path.abspath(tq.__file__))
+    exe = tmp_path / "abi_from_c"
+    build = subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                            "-I", os.path.join(root, "include"),
+                            os.path.join(root, "tests", "native", "abi_from_c.c"),
+                            "-L", pkg, "-ltq", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
+                           capture_output=True, text=True, timeout=120)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    got = {ln.split()[0]: ln.split()[1:] for ln in run.stdout.splitlines() if ln.strip()}
+    cb = tq.Codebook(128, 3, 4, qjl=True, seed=42)
+    t = cb.tables()
+    assert got["init"] == ["0"] and got["tables"] == ["0"]
+    lay = cb.layout
+    assert got["layout"] == [str(x) for x in (lay.k_code_bytes, lay.v_code_bytes, lay.k_sign_bytes,
+                                              lay.norm_halves)]
+    assert np.array_equal(np.array(got["k_centroids"], np.float32), t["k_centroids"].numpy())
+    assert [int(x) for x in got["signs1"]] == t["signs1"].tolist()[:16]
+    assert int(got["decode_ws"][0]) == tq.tq_decode_workspace_bytes(cb, 32, 32, 8, 65536)
+    assert int(got["lut_ws"][0]) == tq.tq_lut_matmul_workspace_bytes(cb, 16384, 8192, 16)
+    assert got["rejected"][0] == str(tq.TQ_ERR_INVALID) and "cache is NULL" in " ".join(got["rejected"])
+
+
 def test_library_exports_every_declared_symbol():
     names = _declared()
     assert set(names) == set(tq.EXPORTS)
