@@ -22,8 +22,9 @@ def _declared():
 
 
 def test_plain_c_client(tmp_path):
-    """include/tq.h compiles as strict C99 and a C program linked against
-    libtq.so gets the same answers as the Python binding (host-only calls)."""
+    """include/tq.h compiles as strict C99 and as C++17, and a program linked
+    against libtq.so gets the same answers as the Python binding (host-only
+    calls)."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
@@ -31,16 +32,22 @@ def test_plain_c_client(tmp_path):
         pytest.skip("no C compiler")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     pkg = os.path.dirname(os.path.abspath(tq.__file__))
-    exe = tmp_path / "abi_from_c"
-    build = subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
-                            "-I", os.path.join(root, "include"),
-                            os.path.join(root, "tests", "native", "abi_from_c.c"),
-                            "-L", pkg, "-ltq", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
-                           capture_output=True, text=True, timeout=120)
-    assert build.returncode == 0, build.stderr
-    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
-    assert run.returncode == 0, run.stdout + run.stderr
-    got = {ln.split()[0]: ln.split()[1:] for ln in run.stdout.splitlines() if ln.strip()}
+    src = os.path.join(root, "tests", "native", "abi_from_c.c")
+    outputs = []
+    # as C99, and the same source as C++ (the header's extern "C" linkage)
+    for lang, std in (("c", "-std=c99"), ("c++", "-std=c++17")):
+        exe = tmp_path / f"abi_from_{lang.replace('+', 'p')}"
+        build = subprocess.run([cc, "-x", lang, std, "-pedantic", "-Wall", "-Wextra", "-Werror",
+                                "-I", os.path.join(root, "include"), src, "-x", "none",
+                                "-L", pkg, "-ltq", f"-Wl,-rpath,{pkg}", "-o", str(exe)]
+                               + (["-lstdc++"] if lang == "c++" else []),
+                               capture_output=True, text=True, timeout=120)
+        assert build.returncode == 0, build.stderr
+        run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+        assert run.returncode == 0, run.stdout + run.stderr
+        outputs.append(run.stdout)
+    assert outputs[0] == outputs[1]
+    got = {ln.split()[0]: ln.split()[1:] for ln in outputs[0].splitlines() if ln.strip()}
     cb = tq.Codebook(128, 3, 4, qjl=True, seed=42)
     t = cb.tables()
     assert got["init"] == ["0"] and got["tables"] == ["0"]
