@@ -61,6 +61,31 @@ def test_plain_c_client(tmp_path):
     assert got["rejected"][0] == str(tq.TQ_ERR_INVALID) and "cache is NULL" in " ".join(got["rejected"])
 
 
+def test_last_error_is_per_thread():
+    """Each thread reads the message of its own last failing call."""
+    import threading
+    cb = tq.Codebook(128, 3, 4)
+    barrier = threading.Barrier(2)
+    seen = {}
+
+    def worker(name, fail):
+        for _ in range(200):
+            fail()
+            barrier.wait()          # the other thread has failed differently in between
+            seen.setdefault(name, set()).add(tq.tq_last_error())
+            barrier.wait()
+
+    fails = {"capacity": lambda: _append(cb, _fake_cache(capacity=40)),
+             "dtype": lambda: _append(cb, _fake_cache(), dtype=7)}
+    threads = [threading.Thread(target=worker, args=(n, f)) for n, f in fails.items()]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=60)
+    assert len(seen["capacity"]) == 1 and "multiple of 16" in next(iter(seen["capacity"]))
+    assert len(seen["dtype"]) == 1 and "unknown dtype" in next(iter(seen["dtype"]))
+
+
 def test_library_exports_every_declared_symbol():
     names = _declared()
     assert set(names) == set(tq.EXPORTS)
