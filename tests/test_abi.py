@@ -146,6 +146,14 @@ def test_codebook_init_null_arguments():
     h = C.c_void_p()
     assert tq.lib.tq_codebook_init(None, C.byref(h), None) == tq.TQ_ERR_INVALID
     assert tq.lib.tq_codebook_init(C.byref(params), None, None) == tq.TQ_ERR_INVALID
+    # a NULL layout is allowed; any table buffer may be NULL; tq_free(NULL) is a no-op
+    assert tq.lib.tq_codebook_init(C.byref(params), C.byref(h), None) == tq.TQ_OK and h.value
+    assert tq.lib.tq_codebook_tables(h, None, None, None, None, None, None) == tq.TQ_OK
+    kc = (C.c_float * 8)()
+    assert tq.lib.tq_codebook_tables(h, kc, None, None, None, None, None) == tq.TQ_OK
+    assert list(kc) == tq.Codebook(128, 3, 4).tables()["k_centroids"].tolist()
+    tq.lib.tq_free(h)
+    tq.lib.tq_free(None)
 
 
 def test_affine_layout_matches_the_pages_memory_table(golden):
