@@ -93,7 +93,7 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(tq.lib, n), n
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kb,vb", [(2, 2), (3, 4), (4, 4), (2, 3)])
 @pytest.mark.parametrize("seed", [0, 1234567, 2**64 - 1])
 def test_tables_equal_oracle_bit_for_bit(d, kb, vb, seed):
@@ -107,7 +107,7 @@ def test_tables_equal_oracle_bit_for_bit(d, kb, vb, seed):
     assert np.array_equal(t["signs2"].numpy(), o.rotation_signs(seed, d, second=True))
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kb,vb", [(2, 2), (3, 4), (4, 4), (2, 3), (3, 3)])
 def test_sphere_tables_equal_oracle_bit_for_bit(d, kb, vb):
     """The host solves the sphere codebook with its own integration (Gauss-Legendre
