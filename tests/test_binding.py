@@ -1,6 +1,9 @@
 """Host-side checks of the Python binding (CPU only: every call below is
 rejected by the binding's own argument checks before the library is reached,
 or touches host memory only)."""
+import os
+import re
+
 import pytest
 import torch
 
@@ -74,3 +77,26 @@ def test_output_buffer_checks():
                 torch.zeros(2, 128, 4).transpose(1, 2)):
         with pytest.raises(ValueError, match="out must be"):
             tq._check_out("decode", bad, (2, 4, 128))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without libtq.so next to it the binding refuses to import: there is no
+    fallback implementation to drop back to."""
+    import importlib.util
+    import shutil
+    src = os.path.join(os.path.dirname(os.path.abspath(tq.__file__)), "tq.py")
+    shutil.copy(src, tmp_path / "tq.py")
+    spec = importlib.util.spec_from_file_location("tq_without_library", tmp_path / "tq.py")
+    with pytest.raises(ImportError, match="libtq.so is not built"):
+        spec.loader.exec_module(importlib.util.module_from_spec(spec))
+
+
+def test_product_never_imports_the_oracle():
+    """The oracle is test infrastructure: no product source names it."""
+    pkg = os.path.dirname(os.path.abspath(tq.__file__))
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "tq_oracle" not in text, f
