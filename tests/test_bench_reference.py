@@ -62,3 +62,13 @@ def test_clock_summary_parses_nvidia_smi_lines():
     assert s["reasons"] == ["sw_power_cap"]
     c.out = ""
     assert c.summary()["reasons"] == ["unavailable"]
+
+
+def test_other_ranks_print_nothing():
+    """Under torchrun every rank but 0 exits 0 without work or output."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "3", "--warmup", "3", "--gpus", "2"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
