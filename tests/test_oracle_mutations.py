@@ -15,6 +15,7 @@ from __future__ import annotations
 import inspect
 import itertools
 import signal
+import threading
 
 import pytest
 
@@ -150,19 +151,24 @@ class _TooSlow(Exception):
 
 def _caught(fn, kw, seconds=30) -> bool:
     """True when the pin fails (an assertion, an error, or no answer within
-    ``seconds``: an iteration that stops converging counts as caught)."""
+    ``seconds``: an iteration that stops converging counts as caught; the
+    limit needs SIGALRM and the main thread, and is skipped without them)."""
+    timed = hasattr(signal, "SIGALRM") and threading.current_thread() is threading.main_thread()
+
     def alarm(*_):
         raise _TooSlow()
-    old = signal.signal(signal.SIGALRM, alarm)
-    signal.alarm(seconds)
+    if timed:
+        old = signal.signal(signal.SIGALRM, alarm)
+        signal.alarm(seconds)
     try:
         fn(**kw)
         return False
     except Exception:
         return True
     finally:
-        signal.alarm(0)
-        signal.signal(signal.SIGALRM, old)
+        if timed:
+            signal.alarm(0)
+            signal.signal(signal.SIGALRM, old)
 
 
 @pytest.mark.parametrize("case,name,old,new,modules", MUTANTS, ids=[m[0] for m in MUTANTS])
